@@ -1,0 +1,51 @@
+"""The seeded input generator: stream order, chunking and bf16 rounding (CPU only)."""
+import numpy as np
+import torch
+
+from exact_io_aware_68_b200.inputs import (bf16_bits_to_f64, f32_to_bf16_bits, make_inputs,
+                                           sampled_rows)
+from exact_io_aware_68_b200.workloads import WORKLOADS
+
+
+def test_head_chunking_matches_one_draw():
+    w = WORKLOADS["bf16_4x16x1024x64"]
+    x = make_inputs(w, N=32, B=2, H=3)
+    rng = np.random.default_rng(w.seed)
+    for name in ("q", "k", "v", "do"):
+        full = rng.standard_normal((2, 3, 32, w.d)) * w.factor
+        np.testing.assert_array_equal(x[name], f32_to_bf16_bits(full.astype(np.float32)))
+
+
+def test_bf16_rounding_matches_torch():
+    x = np.random.default_rng(0).standard_normal(1 << 16).astype(np.float32)
+    x[:4] = [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 3.0e38]   # ties and a large value
+    mine = f32_to_bf16_bits(x)
+    theirs = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(mine, theirs)
+    back = bf16_bits_to_f64(mine)
+    np.testing.assert_array_equal(back, torch.from_numpy(x).to(torch.bfloat16).double().numpy())
+
+
+def test_exact_values_and_key_lengths():
+    w = WORKLOADS["bf16_keypad_dropout_16x16x512x64"]
+    x = make_inputs(w, H=2)
+    np.testing.assert_array_equal(bf16_bits_to_f64(x["q"]), x["q64"])
+    assert x["key_lens"].shape == (16,) and x["key_lens"].min() >= 256 and x["key_lens"].max() <= 512
+    y = make_inputs(w, H=2)
+    np.testing.assert_array_equal(x["key_lens"], y["key_lens"])
+    f = make_inputs(WORKLOADS["fp32_1x1x128x64"], with_do=False)
+    assert f["q"].dtype == np.float32 and "do" not in f
+
+
+def test_headline_scale_factor():
+    w = WORKLOADS["bf16_causal_2x16x4096x128"]
+    x = make_inputs(w, N=64, B=1, H=1)
+    ref = np.random.default_rng(w.seed).standard_normal((1, 1, 64, 128)) * 0.5
+    np.testing.assert_array_equal(x["q"], f32_to_bf16_bits(ref.astype(np.float32)))
+
+
+def test_sampled_rows_are_distinct_and_seeded():
+    r = sampled_rows(4, 3, 65536, 256)
+    assert len(set(r.tolist())) == 256 and r.max() < 65536
+    np.testing.assert_array_equal(r, sampled_rows(4, 3, 65536, 256))
+    assert not np.array_equal(r, sampled_rows(4, 2, 65536, 256))
