@@ -1,0 +1,520 @@
+// Exact attention backward for sm_100a, recomputing each probability block from Q, K and the
+// saved per-row logsumexp instead of storing P ("48 FlashAttention", block "Backward — тоже без
+// N×N"; "Flash Attention：如何通过硬件感知优化重塑注意力机制的未来", section 2.2: keep only the
+// softmax normalisers and rebuild the attention weights on demand).  Gradients are the exact
+// derivatives of O = dropout(softmax(mask(tau Q K^T))) V:
+//   dV = Pt^T dO,  dPt = dO V^T,  dP = dPt * Z/(1-p),  D_i = rowsum(dO * O)_i,
+//   dS = P * (dP - D),  dQ = tau dS K,  dK = tau dS^T Q.
+//
+// Three launches:
+//   fa_bwd_prep_kernel    D = rowsum(dO * O) in fp32, clears the fp32 dQ accumulator
+//   fa_bwd_sm100_kernel   one CTA per (b, h, 128-key tile), K and V resident, loop over query
+//                         tiles; S^T, dP^T, dV, dK, dQ on tcgen05; dQ added into the fp32
+//                         accumulator with vector atomics (fp32 gradient accumulation, as the
+//                         mixed-precision advice in section 3.2 of the same blog post asks)
+//   fa_bwd_dq_kernel      dQ = bf16(tau * accumulator)
+//
+// Main kernel roles (10 warps):
+//   warps 0-3  compute: thread r owns key row r (TMEM lane r): P^T = exp2(S^T*tau*log2e - lse2),
+//              masks, dropout, writes (P*Z)^T (bf16) to TMEM (dV takes 1/(1-p) at the end); dS^T = P^T * (dP^T - D) to TMEM (bf16)
+//              and dS to shared memory (MN-major, the A operand of dQ = dS K); dV epilogue
+//   warps 4-7  dQ: read the 128 x D dQ tile from TMEM, atomically add to the accumulator; dK epilogue
+//   warp 8     producer: TMA K, V once; Q, dO per query tile (STAGES deep); lse and D per tile
+//   warp 9     MMA issuer
+// TMEM (512 columns): ST [0,128) S^T then P~^T in [0,64); DPT [128,256) dP^T then dS^T in
+// [128,192); dV [256,256+D); dK [256+D,256+2D).  dQ: D=64 -> [384,448); D=128 -> the upper
+// halves [64,128) and [192,256), so the next S^T / dP^T waits until dQ has been read.
+#pragma once
+#include <cuda_bf16.h>
+#include "sm100.cuh"
+#include "dropout_hash.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const __nv_bfloat16* o;      // [B,H,N,D]   (prep)
+  const __nv_bfloat16* dO;     // [B,H,N,D]   (prep)
+  const float* lse;            // [B,H,N]
+  float* dvec;                 // [B,H,N]     D = rowsum(dO * O)
+  float* dq_acc;               // [B,H,N,D]   fp32
+  __nv_bfloat16* dq;           // [B,H,N,D]
+  __nv_bfloat16* dk;           // [B,H,N,D]
+  __nv_bfloat16* dv;           // [B,H,N,D]
+  const int32_t* key_lens;     // [B] or null
+  int B, H, N;
+  int n_tiles;                 // ceil(N / 128)
+  int causal;
+  float scale;                 // tau
+  float scale_log2;            // tau * log2(e)
+  int dropout;
+  uint32_t drop_thr;
+  float drop_scale;
+  uint64_t seed;
+  uint64_t wait_ns;
+};
+
+constexpr float kLog2e = 1.4426950408889634074f;
+
+// ----------------------------------------------------------------------------- prep
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
+  constexpr int TPR = D / 8;                       // threads per row, 8 elements (16 bytes) each
+  const uint64_t rows = uint64_t(p.B) * p.H * p.N;
+  const uint64_t t = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint64_t row = t / TPR;
+  const int part = int(t % TPR);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 ov = reinterpret_cast<const uint4*>(p.o + row * D)[part];
+    const uint4 gv = reinterpret_cast<const uint4*>(p.dO + row * D)[part];
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = __bfloat1622float2(o2[e]);
+      const float2 c = __bfloat1622float2(g2[e]);
+      acc = fmaf(a.x, c.x, acc);
+      acc = fmaf(a.y, c.y, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && part == 0) p.dvec[row] = acc;
+}
+
+// ----------------------------------------------------------------------------- dq convert
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
+  const uint64_t n8 = uint64_t(p.B) * p.H * p.N * D / 8;
+  for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += uint64_t(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[2 * i];
+    const float4 c = reinterpret_cast<const float4*>(p.dq_acc)[2 * i + 1];
+    uint4 r;
+    r.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
+    r.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
+    r.z = pack_bf16x2(c.x * p.scale, c.y * p.scale);
+    r.w = pack_bf16x2(c.z * p.scale, c.w * p.scale);
+    reinterpret_cast<uint4*>(p.dq)[i] = r;
+  }
+}
+
+// ----------------------------------------------------------------------------- main
+template <int D>
+struct BwdLayout {
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int SUB = 128 * 128;
+  static constexpr int STAGES = (D == 128) ? 2 : 3;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + TILE;
+  static constexpr int Q_OFF = V_OFF + TILE;
+  static constexpr int DO_OFF = Q_OFF + STAGES * TILE;
+  static constexpr int DS_OFF = DO_OFF + STAGES * TILE;      // 128 keys x 128 queries bf16, 2 panels
+  static constexpr int STAT_OFF = DS_OFF + 2 * SUB;           // per stage: lse2[128], D[128]
+  static constexpr int BAR_OFF = STAT_OFF + STAGES * 1024;
+  // kv_full, q_full[S], do_full[S], stat_full[S], q_empty[S], s_full, dp_full, p_full, ds_full,
+  // dq_full, dq_empty, fin
+  static constexpr int NBARS = 1 + 4 * STAGES + 7;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int ST_COL = 0, DPT_COL = 128, DV_COL = 256, DK_COL = 256 + D;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
+  static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using L = BwdLayout<D>;
+  constexpr int STAGES = L::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (tid == 0) record_status(kStatusBadSmemAlign);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* do_full = q_full + STAGES;
+  uint64_t* stat_full = do_full + STAGES;
+  uint64_t* q_empty = stat_full + STAGES;
+  uint64_t* s_full = q_empty + STAGES;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* p_full = dp_full + 1;
+  uint64_t* ds_full = p_full + 1;
+  uint64_t* dq_full = ds_full + 1;
+  uint64_t* dq_empty = dq_full + 1;
+  uint64_t* fin = dq_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
+
+  // ---- work item: (b, h, key tile kt); heavy causal tiles (small kt) first
+  const int kt = int(blockIdx.x);
+  const int bh = blockIdx.y;
+  const int b = bh / p.H;
+  const int k0 = kt * 128;
+  int kv_end = p.N;
+  if (p.key_lens != nullptr) kv_end = min(kv_end, max(p.key_lens[b], 0));
+  const int q_first = p.causal ? kt : 0;
+  const int n_iter = (k0 < kv_end) ? (p.n_tiles - q_first) : 0;
+
+  if (tid == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&do_full[s], 1);
+      mbar_init(&stat_full[s], 32);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(ds_full, 4);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 4);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{p.wait_ns, abort_flag};
+  const uint64_t row_base = uint64_t(bh) * uint64_t(p.N);
+
+  if (warp == 8) {
+    // =========================================================== producer
+    int issued = 0;
+    if (n_iter > 0) {
+      if (lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(smem + L::K_OFF + c * L::SUB, &tm_k, kv_full, c * 64, k0, bh);
+          tma_load_3d(smem + L::V_OFF + c * L::SUB, &tm_v, kv_full, c * 64, k0, bh);
+        }
+      }
+      for (int t = 0; t < n_iter; ++t) {
+        const int st = t % STAGES;
+        const int qrow0 = (q_first + t) * 128;
+        if (t >= STAGES && !warp_wait(&q_empty[st], ((t / STAGES) - 1) & 1, wc)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full[st], L::TILE);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + L::Q_OFF + st * L::TILE + c * L::SUB, &tm_q, &q_full[st], c * 64, qrow0, bh);
+          mbar_arrive_expect_tx(&do_full[st], L::TILE);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + L::DO_OFF + st * L::TILE + c * L::SUB, &tm_do, &do_full[st], c * 64, qrow0, bh);
+        }
+        // per-query statistics of this tile: lse in the exp2 domain and D
+        float* st_l = stat + st * 256;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = lane * 4 + e;
+          const int q = qrow0 + c;
+          float lv = 0.f, dv = 0.f;
+          if (q < p.N) {
+            lv = p.lse[row_base + q] * kLog2e;
+            dv = p.dvec[row_base + q];
+          }
+          st_l[c] = lv;
+          st_l[128 + c] = dv;
+        }
+        mbar_arrive(&stat_full[st]);
+        issued = t + 1;
+      }
+      if (lane == 0) {
+        mbar_drain(kv_full, 0, p.wait_ns);
+        for (int t = max(0, issued - STAGES); t < issued; ++t) {
+          mbar_drain(&q_full[t % STAGES], (t / STAGES) & 1, p.wait_ns);
+          mbar_drain(&do_full[t % STAGES], (t / STAGES) & 1, p.wait_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // =========================================================== MMA issuer
+    if (lane == 0 && n_iter > 0) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (or V) K-major, Q (or dO) K-major
+      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // A in TMEM, B MN-major
+      constexpr uint32_t kIdQ = idesc_bf16(128, 64, true, true);      // dS MN-major, K MN-major, N = 64
+      const uint32_t k_base = smem_u32(smem + L::K_OFF);
+      const uint32_t v_base = smem_u32(smem + L::V_OFF);
+      const uint32_t ds_base = smem_u32(smem + L::DS_OFF);
+      bool ok = mbar_wait(kv_full, 0, wc);
+      for (int t = 0; ok && t < n_iter; ++t) {
+        const int st = t % STAGES;
+        const uint32_t sp = (t / STAGES) & 1;
+        const uint32_t q_base = smem_u32(smem + L::Q_OFF + st * L::TILE);
+        const uint32_t do_base = smem_u32(smem + L::DO_OFF + st * L::TILE);
+        if (!mbar_wait(&q_full[st], sp, wc)) { ok = false; break; }
+        if (D == 128 && t >= 1 && !mbar_wait(dq_empty, (t - 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        // S^T = K Q^T  (M = 128 keys, N = 128 queries, K = D)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
+          mma_ss(tmem + L::ST_COL, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(q_base + off, 16, 1024), kIdS,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+        // dP^T = V dO^T
+        if (!mbar_wait(&do_full[st], sp, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
+          mma_ss(tmem + L::DPT_COL, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(do_base + off, 16, 1024),
+                 kIdS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dp_full);
+        // dV += P~^T dO   (A = P~^T in TMEM, B = dO MN-major: N = D, K = queries)
+        if (!mbar_wait(p_full, t & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_sw128(do_base + kk * 2048, L::SUB, 1024), kIdG,
+                 (t > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q
+        if (!mbar_wait(ds_full, t & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::DK_COL, tmem + L::DPT_COL + kk * 8, sdesc_sw128(q_base + kk * 2048, L::SUB, 1024), kIdG,
+                 (t > 0 || kk > 0) ? 1u : 0u);
+        // dQ_tile = dS K   (M = 128 queries, K = 128 keys, N = 64 per panel of D)
+        if (D == 64 && t >= 1 && !mbar_wait(dq_empty, (t - 1) & 1, wc)) { ok = false; break; }
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          const uint32_t dq_col = (D == 64) ? 384u : (h == 0 ? 64u : 192u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + dq_col, sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024),
+                   sdesc_sw128(k_base + h * L::SUB + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(dq_full);
+        mma_commit(&q_empty[st]);
+      }
+      mma_commit(fin);
+      mbar_drain(fin, 0, p.wait_ns);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // =========================================================== compute (key row r)
+    const int r = tid;
+    const int key = k0 + r;
+    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    uint8_t* ds_smem = smem + L::DS_OFF;
+    for (int t = 0; t < n_iter; ++t) {
+      const int st = t % STAGES;
+      const int qrow0 = (q_first + t) * 128;
+      const float* st_l = stat + st * 256;
+      const bool need_mask = (k0 + 128 > kv_end) || (qrow0 + 128 > p.N) || (p.causal && q_first + t == kt);
+      if (!warp_wait(s_full, t & 1, wc)) { ok = false; break; }
+      if (!warp_wait(&stat_full[st], (t / STAGES) & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      float pr[128];                 // P^T row (undropped), fp32
+      uint32_t keep_bits[4] = {0u, 0u, 0u, 0u};
+      const uint64_t drop_col0 = (row_base + uint64_t(qrow0)) * uint64_t(p.N) + uint64_t(key);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sr[32];
+        tmem_ld32(lane_base + L::ST_COL + ch * 32, sr);
+        tmem_ld_wait();
+        reg_fence32(sr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = ch * 32 + e;
+          float pv = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -st_l[c]));
+          if (need_mask) {
+            const int q = qrow0 + c;
+            if (key >= kv_end || q >= p.N || (p.causal && key > q)) pv = 0.f;
+          }
+          pr[c] = pv;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = ch * 32 + 2 * e;
+          float a = pr[c], bb = pr[c + 1];
+          if (p.dropout) {
+            // element (query i = qrow0 + c, key j = key): ctr = (bh*N + i)*N + j
+            const uint64_t ctr = drop_col0 + uint64_t(c) * uint64_t(p.N);
+            const bool ka = dropout_keep(p.seed, ctr, p.drop_thr);
+            const bool kb = dropout_keep(p.seed, ctr + uint64_t(p.N), p.drop_thr);
+            keep_bits[ch] |= (ka ? 1u : 0u) << (2 * e);
+            keep_bits[ch] |= (kb ? 1u : 0u) << (2 * e + 1);
+            a = ka ? a : 0.f;      // P * Z; dV takes the 1/(1-p) factor in its fp32 epilogue
+            bb = kb ? bb : 0.f;
+          }
+          pk[e] = pack_bf16x2(a, bb);
+        }
+        // P~^T columns [16ch, 16ch+16) overlay score columns already read
+        tmem_st16(lane_base + L::ST_COL + ch * 16, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+
+      // ---- dS^T = P^T * (dP^T - D)
+      if (!warp_wait(dp_full, t & 1, wc)) { ok = false; break; }
+      // the previous dQ MMA has finished reading the dS tile in shared memory
+      if (t >= 1 && !warp_wait(dq_full, (t - 1) & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t dr[32];
+        tmem_ld32(lane_base + L::DPT_COL + ch * 32, dr);
+        tmem_ld_wait();
+        reg_fence32(dr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = ch * 32 + 2 * e;
+          float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
+          if (p.dropout) {
+            dpa = ((keep_bits[ch] >> (2 * e)) & 1u) ? dpa * p.drop_scale : 0.f;
+            dpb = ((keep_bits[ch] >> (2 * e + 1)) & 1u) ? dpb * p.drop_scale : 0.f;
+          }
+          const float dsa = pr[c] * (dpa - st_l[128 + c]);
+          const float dsb = pr[c + 1] * (dpb - st_l[128 + c + 1]);
+          pk[e] = pack_bf16x2(dsa, dsb);
+        }
+        tmem_st16(lane_base + L::DPT_COL + ch * 16, pk);
+        // dS (queries contiguous) into the 128-byte-swizzled panel: row = key r, 16-byte chunks
+        const int panel = ch >> 1;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const int chunk = (ch & 1) * 4 + v4;   // 8 queries per 16-byte chunk
+          uint4* dst = reinterpret_cast<uint4*>(ds_smem + panel * L::SUB + r * 128 + ((chunk ^ (r & 7)) << 4));
+          *dst = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
+    }
+    // ---- dV epilogue
+    if (n_iter == 0) {
+      if (key < p.N) {
+        uint4* dst = reinterpret_cast<uint4*>(p.dv + (row_base + key) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+      }
+    } else if (ok && warp_wait(fin, 0, wc)) {
+      tc_fence_after();
+      const float s = p.dropout ? p.drop_scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t vr[32];
+        tmem_ld32(lane_base + L::DV_COL + c * 32, vr);
+        tmem_ld_wait();
+        reg_fence32(vr);
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(p.dv + (row_base + key) * D + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(vr[8 * e]) * s, __uint_as_float(vr[8 * e + 1]) * s),
+                                pack_bf16x2(__uint_as_float(vr[8 * e + 2]) * s, __uint_as_float(vr[8 * e + 3]) * s),
+                                pack_bf16x2(__uint_as_float(vr[8 * e + 4]) * s, __uint_as_float(vr[8 * e + 5]) * s),
+                                pack_bf16x2(__uint_as_float(vr[8 * e + 6]) * s, __uint_as_float(vr[8 * e + 7]) * s));
+        }
+      }
+    }
+  } else {
+    // =========================================================== dQ readout + dK epilogue (warps 4-7)
+    const int quarter = warp - 4;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    bool ok = true;
+    for (int t = 0; t < n_iter; ++t) {
+      const int q = (q_first + t) * 128 + r;
+      if (!warp_wait(dq_full, t & 1, wc)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t g[D];
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        const uint32_t col = (D == 64) ? 384u : (h == 0 ? 64u : 192u);
+        tmem_ld32(lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&g[h * 64]));
+        tmem_ld32(lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[h * 64 + 32]));
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int h = 0; h < D / 32; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&g[h * 32]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_empty);
+      if (q < p.N) {
+        float4* dst = reinterpret_cast<float4*>(p.dq_acc + (row_base + q) * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c)
+          atomicAdd(dst + c, make_float4(__uint_as_float(g[4 * c]), __uint_as_float(g[4 * c + 1]),
+                                         __uint_as_float(g[4 * c + 2]), __uint_as_float(g[4 * c + 3])));
+      }
+    }
+    const int key = k0 + r;
+    if (n_iter == 0) {
+      if (key < p.N) {
+        uint4* dst = reinterpret_cast<uint4*>(p.dk + (row_base + key) * D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+      }
+    } else if (ok && warp_wait(fin, 0, wc)) {
+      tc_fence_after();
+      const float s = p.scale;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t kr[32];
+        tmem_ld32(lane_base + L::DK_COL + c * 32, kr);
+        tmem_ld_wait();
+        reg_fence32(kr);
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(p.dk + (row_base + key) * D + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(kr[8 * e]) * s, __uint_as_float(kr[8 * e + 1]) * s),
+                                pack_bf16x2(__uint_as_float(kr[8 * e + 2]) * s, __uint_as_float(kr[8 * e + 3]) * s),
+                                pack_bf16x2(__uint_as_float(kr[8 * e + 4]) * s, __uint_as_float(kr[8 * e + 5]) * s),
+                                pack_bf16x2(__uint_as_float(kr[8 * e + 6]) * s, __uint_as_float(kr[8 * e + 7]) * s));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,366 @@
+// The C ABI declared in include/fa.h: argument validation, TMA descriptor encoding and the
+// kernel launches.  The kernels live in the headers included below; this is the library's
+// single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "bwd_sm100.cuh"
+#include "fwd_sm100.cuh"
+#include "simt_f32.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+fa_status fail(fa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+uint64_t default_wait_ns() {
+  const char* e = std::getenv("FA_WAIT_LIMIT_MS");
+  if (e != nullptr) {
+    const long long ms = std::atoll(e);
+    if (ms > 0) return uint64_t(ms) * 1000000ull;
+  }
+  return 2000000000ull;
+}
+std::atomic<uint64_t> g_wait_ns{default_wait_ns()};
+std::atomic<int> g_debug_flags{0};
+
+// cuTensorMapEncodeTiled from the driver, fetched through the runtime (no -lcuda needed).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D view {d, N, B*H} of a bf16 [B,H,N,d] tensor, loaded as 64 x 128 x 1 boxes with the
+// 128-byte swizzle; rows past N (the ragged last tile) read as zeros.
+fa_status make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, const char* name) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * cuuint64_t(d) * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", name, int(r));
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int H, int N, int d, float scale, float dropout_p, bool bf16) {
+  if (B < 1 || H < 1 || N < 1) return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1 (got %d, %d, %d)", B, H, N);
+  if (int64_t(B) * H > 65535) return fail(FA_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", (long long)B * H);
+  if (int64_t(N) > (int64_t(1) << 30)) return fail(FA_ERR_UNSUPPORTED, "N = %d is too large", N);
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: %s supports d in {64, 128}", d, bf16 ? "bf16" : "fp32");
+  if (!std::isfinite(scale) || !(scale > 0.f)) return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!(dropout_p >= 0.f) || !(dropout_p < 1.f)) return fail(FA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
+  return FA_OK;
+}
+
+#define FA_CHECK_PTR(p)                                                                      \
+  do {                                                                                       \
+    if ((p) == nullptr) return fail(FA_ERR_INVALID_ARG, "%s is NULL", #p);                   \
+    if (!aligned16(p)) return fail(FA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);     \
+  } while (0)
+
+fa_status launch_status(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return FA_OK;
+}
+
+uint32_t drop_threshold(float p) {
+  const double t = std::floor(double(p) * 4294967296.0);
+  return uint32_t(t > 4294967295.0 ? 4294967295.0 : t);
+}
+
+struct Workspace {
+  float* dq_acc;
+  float* dvec;
+};
+size_t ws_dq_bytes(int B, int H, int N, int d) {
+  return (size_t(B) * H * N * d * 4 + 255) & ~size_t(255);
+}
+size_t ws_total_bytes(int B, int H, int N, int d) {
+  return ws_dq_bytes(B, H, N, d) + ((size_t(B) * H * N * 4 + 255) & ~size_t(255));
+}
+fa_status check_workspace(void* ws, size_t bytes, int B, int H, int N, int d, Workspace* out) {
+  if (ws == nullptr) return fail(FA_ERR_INVALID_ARG, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(FA_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  const size_t need = ws_total_bytes(B, H, N, d);
+  if (bytes < need) return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", bytes, need);
+  out->dq_acc = static_cast<float*>(ws);
+  out->dvec = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_dq_bytes(B, H, N, d));
+  return FA_OK;
+}
+
+template <typename K>
+fa_status set_smem(K kernel, int bytes) {
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+template <int D>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
+                     cudaStream_t s) {
+  using L = fa::FwdLayout<D>;
+  fa_status st = set_smem(fa::fa_fwd_sm100_kernel<D>, L::BYTES);
+  if (st != FA_OK) return st;
+  const dim3 grid(p.n_qtiles, p.B * p.H);
+  fa::fa_fwd_sm100_kernel<D><<<grid, 192, L::BYTES, s>>>(mq, mk, mv, p);
+  return launch_status("fa_fwd kernel launch");
+}
+
+template <int D>
+fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                          const fa::BwdParams& p, cudaStream_t s) {
+  using L = fa::BwdLayout<D>;
+  fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D>, L::BYTES);
+  if (st != FA_OK) return st;
+  const dim3 grid(p.n_tiles, p.B * p.H);
+  fa::fa_bwd_sm100_kernel<D><<<grid, 320, L::BYTES, s>>>(mq, mk, mv, mdo, p);
+  return launch_status("fa_bwd main kernel launch");
+}
+
+fa::BwdParams bwd_params(int B, int H, int N, float scale, int causal, const int32_t* key_lens, float dropout_p,
+                         uint64_t seed, const Workspace& w) {
+  fa::BwdParams p{};
+  p.lse = nullptr;
+  p.dvec = w.dvec;
+  p.dq_acc = w.dq_acc;
+  p.key_lens = key_lens;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_tiles = (N + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.dropout = dropout_p > 0.f ? 1 : 0;
+  p.drop_thr = drop_threshold(dropout_p);
+  p.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
+  p.seed = seed;
+  p.wait_ns = g_wait_ns.load();
+  return p;
+}
+
+unsigned grid_for(uint64_t work, unsigned per_block) {
+  const uint64_t g = (work + per_block - 1) / per_block;
+  return unsigned(g < 1 ? 1 : (g > (1u << 30) ? (1u << 30) : g));
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream) {
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, true);
+  if (st != FA_OK) return st;
+  FA_CHECK_PTR(q);
+  FA_CHECK_PTR(k);
+  FA_CHECK_PTR(v);
+  FA_CHECK_PTR(o);
+  FA_CHECK_PTR(lse);
+  CUtensorMap mq, mk, mv;
+  if ((st = make_tile_map(&mq, q, B * H, N, d, "q")) != FA_OK) return st;
+  if ((st = make_tile_map(&mk, k, B * H, N, d, "k")) != FA_OK) return st;
+  if ((st = make_tile_map(&mv, v, B * H, N, d, "v")) != FA_OK) return st;
+  fa::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.key_lens = key_lens;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_qtiles = (N + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.dropout = dropout_p > 0.f ? 1 : 0;
+  p.drop_thr = drop_threshold(dropout_p);
+  p.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
+  p.seed = seed;
+  p.wait_ns = g_wait_ns.load();
+  p.debug_flags = g_debug_flags.load();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd<64>(mq, mk, mv, p, s) : launch_fwd<128>(mq, mk, mv, p, s);
+}
+
+fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
+                     float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream) {
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, false);
+  if (st != FA_OK) return st;
+  FA_CHECK_PTR(q);
+  FA_CHECK_PTR(k);
+  FA_CHECK_PTR(v);
+  FA_CHECK_PTR(o);
+  FA_CHECK_PTR(lse);
+  fa::F32Params p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.key_lens = key_lens;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.dropout = dropout_p > 0.f ? 1 : 0;
+  p.drop_thr = drop_threshold(dropout_p);
+  p.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
+  p.seed = seed;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dim3 grid((N + 127) / 128, B * H);
+  if (d == 64)
+    fa::fa_fwd_f32_kernel<64><<<grid, 128, 0, s>>>(p);
+  else
+    fa::fa_fwd_f32_kernel<128><<<grid, 128, 0, s>>>(p);
+  return launch_status("fa_fwd_f32 kernel launch");
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  return ws_total_bytes(B, H, N, d);
+}
+
+fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  fa_status st = check_common(B, H, N, d, 1.f, 0.f, true);
+  if (st != FA_OK) return st;
+  FA_CHECK_PTR(o);
+  FA_CHECK_PTR(dO);
+  Workspace w;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
+  fa::BwdParams p = bwd_params(B, H, N, 1.f, 0, nullptr, 0.f, 0, w);
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint64_t threads = uint64_t(B) * H * N * (d / 8);
+  if (d == 64)
+    fa::fa_bwd_prep_kernel<64><<<grid_for(threads, 256), 256, 0, s>>>(p);
+  else
+    fa::fa_bwd_prep_kernel<128><<<grid_for(threads, 256), 256, 0, s>>>(p);
+  return launch_status("fa_bwd_prep kernel launch");
+}
+
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
+                      int B, int H, int N, int d, float scale, int causal, const int32_t* key_lens, float dropout_p,
+                      uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, true);
+  if (st != FA_OK) return st;
+  FA_CHECK_PTR(q);
+  FA_CHECK_PTR(k);
+  FA_CHECK_PTR(v);
+  FA_CHECK_PTR(lse);
+  FA_CHECK_PTR(dO);
+  FA_CHECK_PTR(dk);
+  FA_CHECK_PTR(dv);
+  Workspace w;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_tile_map(&mq, q, B * H, N, d, "q")) != FA_OK) return st;
+  if ((st = make_tile_map(&mk, k, B * H, N, d, "k")) != FA_OK) return st;
+  if ((st = make_tile_map(&mv, v, B * H, N, d, "v")) != FA_OK) return st;
+  if ((st = make_tile_map(&mdo, dO, B * H, N, d, "dO")) != FA_OK) return st;
+  fa::BwdParams p = bwd_params(B, H, N, scale, causal, key_lens, dropout_p, seed, w);
+  p.lse = lse;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd_main<64>(mq, mk, mv, mdo, p, s) : launch_bwd_main<128>(mq, mk, mv, mdo, p, s);
+}
+
+fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  fa_status st = check_common(B, H, N, d, scale, 0.f, true);
+  if (st != FA_OK) return st;
+  FA_CHECK_PTR(dq);
+  Workspace w;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
+  fa::BwdParams p = bwd_params(B, H, N, scale, 0, nullptr, 0.f, 0, w);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint64_t n8 = uint64_t(B) * H * N * d / 8;
+  const unsigned grid = grid_for(n8, 256) > 148u * 16u ? 148u * 16u : grid_for(n8, 256);
+  if (d == 64)
+    fa::fa_bwd_dq_kernel<64><<<grid, 256, 0, s>>>(p);
+  else
+    fa::fa_bwd_dq_kernel<128><<<grid, 256, 0, s>>>(p);
+  return launch_status("fa_bwd_dq_convert kernel launch");
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+                 void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, const int32_t* key_lens,
+                 float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+  FA_CHECK_PTR(dq);
+  fa_status st = fa_bwd_prep(o, dO, B, H, N, d, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  st = fa_bwd_main(q, k, v, lse, dO, dk, dv, B, H, N, d, scale, causal, key_lens, dropout_p, seed, workspace,
+                   workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  return fa_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, uint64_t seed, void* stream) {
+  if (keep == nullptr) return fail(FA_ERR_INVALID_ARG, "keep is NULL");
+  if (B < 1 || H < 1 || N < 1) return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1");
+  if (!(dropout_p >= 0.f) || !(dropout_p < 1.f)) return fail(FA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
+  const uint64_t total = uint64_t(B) * H * N * uint64_t(N);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = grid_for(total, 256) > 148u * 32u ? 148u * 32u : grid_for(total, 256);
+  fa::fa_dropout_mask_kernel<<<grid, 256, 0, s>>>(keep, total, seed, drop_threshold(dropout_p));
+  return launch_status("fa_dropout_mask kernel launch");
+}
+
+fa_status fa_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int code = 0;
+  e = cudaMemcpyFromSymbol(&code, fa::g_fa_device_status, sizeof(int));
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "reading the device status word: %s", cudaGetErrorString(e));
+  if (code == 0) return FA_OK;
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(fa::g_fa_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "clearing the device status word: %s", cudaGetErrorString(e));
+  if (code == fa::kStatusTimeout) return fail(FA_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+  return fail(FA_ERR_INTERNAL, "device status %d (dynamic shared memory not 1024-byte aligned)", code);
+}
+
+const char* fa_get_error(void) { return g_err; }
+
+void fa_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns > 0 ? ns : default_wait_ns()); }
+
+void fa_debug_set_flags(int flags) { g_debug_flags.store(flags); }
+
+const char* fa_version(void) { return "exact-io-aware-attention sm_100a 0.1"; }
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+// fp32 attention forward on the CUDA cores (FFMA, no TF32: a 10-bit-mantissa tensor-core path
+// cannot meet a 1e-5 absolute bar).  Same semantics as the bf16 path: online softmax over key
+// tiles held in shared memory ("48 FlashAttention", block "Tiling и online softmax"), causal and
+// key-padding masks, counter-hash dropout, lse = m + ln l.
+//
+// Also the dropout-mask kernel that writes the keep decisions of the counter hash, so that a
+// test can compare them bit for bit with an independent implementation.
+#pragma once
+#include "dropout_hash.cuh"
+
+namespace fa {
+
+struct F32Params {
+  const float* q;
+  const float* k;
+  const float* v;
+  float* o;
+  float* lse;
+  const int32_t* key_lens;
+  int B, H, N;
+  int causal;
+  float scale;
+  int dropout;
+  uint32_t drop_thr;
+  float drop_scale;
+  uint64_t seed;
+};
+
+// One thread per query row, 128 rows per CTA; K and V staged 32 keys at a time.
+template <int D>
+__global__ void __launch_bounds__(128) fa_fwd_f32_kernel(const F32Params p) {
+  constexpr int KT = 32;
+  __shared__ float ks[KT][D];
+  __shared__ float vs[KT][D];
+  const int bh = blockIdx.y;
+  const int b = bh / p.H;
+  const int row = blockIdx.x * 128 + threadIdx.x;
+  const bool valid = row < p.N;
+  const uint64_t base = uint64_t(bh) * p.N;
+  int kv_end = p.N;
+  if (p.key_lens != nullptr) kv_end = min(kv_end, max(p.key_lens[b], 0));
+  int kv_stop = kv_end;
+  if (p.causal) kv_stop = min(kv_stop, blockIdx.x * 128 + 128);
+
+  float qr[D], acc[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    qr[c] = valid ? p.q[(base + row) * D + c] : 0.f;
+    acc[c] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int j0 = 0; j0 < kv_stop; j0 += KT) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < KT * D; e += 128) {
+      const int jj = e / D, c = e % D;
+      const int j = j0 + jj;
+      ks[jj][c] = j < p.N ? p.k[(base + j) * D + c] : 0.f;
+      vs[jj][c] = j < p.N ? p.v[(base + j) * D + c] : 0.f;
+    }
+    __syncthreads();
+    for (int jj = 0; jj < KT; ++jj) {
+      const int j = j0 + jj;
+      if (j >= kv_end || (p.causal && j > row)) continue;
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < D; ++c) s = fmaf(qr[c], ks[jj][c], s);
+      s *= p.scale;
+      if (s > m) {
+        const float alpha = expf(m - s);
+        l *= alpha;
+#pragma unroll
+        for (int c = 0; c < D; ++c) acc[c] *= alpha;
+        m = s;
+      }
+      float pr = expf(s - m);
+      l += pr;
+      if (p.dropout) {
+        const uint64_t ctr = (base + uint64_t(row)) * uint64_t(p.N) + uint64_t(j);
+        pr = dropout_keep(p.seed, ctr, p.drop_thr) ? pr * p.drop_scale : 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < D; ++c) acc[c] = fmaf(pr, vs[jj][c], acc[c]);
+    }
+  }
+  if (valid) {
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int c = 0; c < D; ++c) p.o[(base + row) * D + c] = acc[c] * inv;
+    p.lse[base + row] = l > 0.f ? m + logf(l) : -INFINITY;
+  }
+}
+
+__global__ void __launch_bounds__(256) fa_dropout_mask_kernel(uint8_t* keep, uint64_t total, uint64_t seed,
+                                                              uint32_t thr) {
+  for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += uint64_t(gridDim.x) * blockDim.x)
+    keep[i] = dropout_keep(seed, i, thr) ? 1 : 0;
+}
+
+}  // namespace fa

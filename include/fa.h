@@ -1,0 +1,131 @@
+/*
+ * exact IO-aware attention for NVIDIA B200 (sm_100a): the C ABI.
+ *
+ * The operation is exact scaled-dot-product attention, one head at a time,
+ *     S = tau * Q K^T,  P = softmax(mask(S)) row by row,  O = dropout(P) V,
+ * as defined in "FlashAttention 的第一原则" (reader.mx), section 2 (Q, K, V and O are N x d,
+ * the N x N intermediates, optional mask and dropout) and section 3.2 (op order matmul, scale,
+ * mask, softmax, dropout), and in "48 FlashAttention" (ml-canon), block "PyTorch FlashAttention
+ * под капотом sdpa" (result identical to softmax(QK^T/sqrt(d)) V).  The forward computes it tile
+ * by tile with an online softmax (same page, block "Tiling и online softmax"): the N x N scores
+ * never reach device memory.  The backward recomputes each probability block from Q, K and the
+ * saved per-row logsumexp (same page, block "Backward — тоже без N×N").
+ *
+ * Conventions for every entry point below.
+ *  - Layouts: q, k, v, o, dO, dq, dk, dv are [B, H, N, d] row-major contiguous (d innermost);
+ *    lse is [B, H, N] fp32, natural log, lse = m + ln(l) over the masked, scaled scores and
+ *    the undropped probabilities.  key_lens is int32 [B] on the device, or NULL.
+ *  - Masks: causal keeps key j <= query i (top-left aligned, self-attention: one N for
+ *    queries and keys); key padding keeps j < key_lens[b] (keys only; every query row is
+ *    computed).  A row with no allowed key gets O = 0, lse = -inf and zero gradients.
+ *  - Dropout (0 <= dropout_p < 1): element (b, h, i, j) is kept when the counter hash
+ *      ctr = ((b*H + h)*N + i)*N + j,  z = seed + (ctr + 1) * 0x9E3779B97F4A7C15 (mod 2^64),
+ *      z = SplitMix64 output mix of z,  keep = (z >> 32) >= min(floor(p * 2^32), 2^32 - 1)
+ *    holds; kept probabilities are multiplied by 1/(1 - p).  The backward must get the same
+ *    (scale, causal, key_lens, dropout_p, seed) as the forward it differentiates.
+ *  - Pointers are DEVICE pointers owned by the caller, 16-byte aligned; the library never
+ *    allocates or frees device memory.  Outputs are overwritten, not accumulated.
+ *  - scale (tau) must be finite and > 0 (1/sqrt(d) is the usual value).
+ *  - bf16 entry points support d in {64, 128}; N >= 1 is arbitrary (tails are zero-filled by
+ *    the tile loads and masked); B*H <= 65535.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  The return value reports argument validation and launch errors only.  Errors
+ *    found on the device (a bounded wait that ran out) are reported by fa_check().
+ *  - On a non-OK return, fa_get_error() describes the failure (thread-local string).
+ */
+#ifndef EXACT_IO_AWARE_FA_H
+#define EXACT_IO_AWARE_FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* a null or misaligned pointer, a size or parameter out of range */
+  FA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement (e.g. d = 96) */
+  FA_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed */
+  FA_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out; its outputs are undefined */
+  FA_ERR_INTERNAL = 5      /* the device reported an inconsistent launch (e.g. shared memory alignment) */
+} fa_status;
+
+/* Forward, bf16.  Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).
+ * q, k, v: bf16 [B,H,N,d].  One kernel launch. */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, float scale, int causal,
+                 const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream);
+
+/* Forward, fp32 throughout (CUDA-core FFMA, no TF32), same semantics and layouts with fp32
+ * q, k, v, o.  d in {64, 128}.  One kernel launch. */
+FA_API fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                     int B, int H, int N, int d, float scale, int causal,
+                     const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream);
+
+/* Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator [B,H,N,d] followed by
+ * D = rowsum(dO * O) fp32 [B,H,N] (each part 256-byte aligned).  0 on invalid sizes. */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/* Backward, bf16.  Given q, k, v, the forward's o and lse, and the upstream gradient dO
+ * (all as produced/consumed by fa_fwd), writes dq, dk, dv (bf16 [B,H,N,d]).
+ * workspace: caller-owned device memory of at least fa_bwd_workspace_size() bytes,
+ * 256-byte aligned, clobbered; it must not be shared by calls that may overlap.
+ * Three kernel launches, in this order: fa_bwd_prep, fa_bwd_main, fa_bwd_dq_convert. */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv,
+                 int B, int H, int N, int d, float scale, int causal,
+                 const int32_t* key_lens, float dropout_p, uint64_t seed,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* The three launches of fa_bwd, exposed separately (same arguments, same workspace) so that a
+ * caller can time or interleave them.  Calling them in order is equivalent to fa_bwd.
+ *  fa_bwd_prep:       D = rowsum(dO * O) into the workspace, clears the dQ accumulator.
+ *  fa_bwd_main:       dK and dV (written), dQ accumulated (fp32) into the workspace.
+ *  fa_bwd_dq_convert: dq = bf16(scale * accumulator). */
+FA_API fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d,
+                      void* workspace, size_t workspace_bytes, void* stream);
+FA_API fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO,
+                      void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                      const int32_t* key_lens, float dropout_p, uint64_t seed,
+                      void* workspace, size_t workspace_bytes, void* stream);
+FA_API fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Writes the dropout keep decisions (1 = kept, 0 = dropped) of every element into
+ * keep (uint8 [B,H,N,N], device).  For testing the counter hash bit for bit. */
+FA_API fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, uint64_t seed,
+                          void* stream);
+
+/* Synchronises `stream`, then reads and clears this device's status word.  Returns
+ * FA_ERR_TIMEOUT if a bounded wait ran out in any kernel since the last check,
+ * FA_ERR_INTERNAL for other device-detected faults, FA_ERR_CUDA if the synchronisation
+ * itself failed, FA_OK otherwise. */
+FA_API fa_status fa_check(void* stream);
+
+/* Description of the last non-OK status returned on the calling thread. */
+FA_API const char* fa_get_error(void);
+
+/* Upper bound, in nanoseconds, on every wait inside the kernels (default 2 s; the
+ * environment variable FA_WAIT_LIMIT_MS overrides the default).  Applies to later launches. */
+FA_API void fa_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook.  Bit 0: the forward's load warp never delivers its first K/V block, so the
+ * consumers' bounded waits run out and fa_check() returns FA_ERR_TIMEOUT.  0 = normal. */
+FA_API void fa_debug_set_flags(int flags);
+
+/* Library version string. */
+FA_API const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_FA_H */

@@ -1,0 +1,78 @@
+"""Shared helpers for the GPU parity tests: upload seeded inputs, run the library, compare
+with the oracle on the same (bf16-rounded) inputs."""
+import numpy as np
+import torch
+
+import oracle
+from exact_io_aware_68_b200 import api
+from exact_io_aware_68_b200.inputs import bf16_bits_to_f64
+
+# Bars from the specification of this library's accuracy (fp32 accumulation everywhere):
+O_MAX_ABS_BF16 = 1e-2      # bf16 outputs vs the fp64 oracle on the bf16-rounded inputs
+O_MAX_ABS_F32 = 1e-5       # fp32 path
+LSE_MAX_ABS = 1e-4
+GRAD_REL_L2 = 1e-2
+
+
+def to_device(x, name):
+    a = x[name]
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return bf16_bits_to_f64(t.cpu().view(torch.int16).numpy().view(np.uint16))
+    return t.double().cpu().numpy()
+
+
+def key_lens_device(x):
+    return None if x["key_lens"] is None else torch.from_numpy(x["key_lens"]).cuda()
+
+
+def run_fwd(x):
+    q, k, v = (to_device(x, n) for n in ("q", "k", "v"))
+    o, lse = api.attention_fwd(q, k, v, x["scale"], x["causal"], key_lens_device(x), x["dropout_p"], x["seed"])
+    api.check()
+    return q, k, v, o, lse
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def bf16_ulp_half(x):
+    """Half a bf16 ulp at |x| (the rounding error bound of the output conversion)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(ax)) - 8)
+
+
+def bf16_product_bound(x, w):
+    """Per-element rounding allowance of a bf16 P.V product for hand-made edge cases.
+
+    P enters the tensor core rounded to bf16 (relative error <= 2^-8: 8 significant bits) and O is
+    stored as bf16 (<= 2^-8 of |O|), so |O_gpu - O| <= 2^-8 (sum_j Pt_ij |V_j| + |O_i|) plus the
+    fp32 accumulation error.  Needs the oracle's P and Z."""
+    O, _, P, Z = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"], w.causal, x["key_lens"], w.dropout_p,
+                                x["seed"], return_p=True)
+    Pt = P if Z is None else P * Z / (1.0 - float(np.float32(w.dropout_p)))
+    return O, 2.0 ** -8 * (np.einsum("bhij,bhjc->bhic", Pt, np.abs(x["v64"])) + np.abs(O))
+
+
+def assert_o_close(o_gpu, o_ref, bar, extra=None):
+    """max |o_gpu - o_ref| <= bar (+ ``extra``, an elementwise allowance for hand-made edge cases,
+    see ``bf16_product_bound``).  An element whose own bf16 output rounding bound exceeds the bar
+    (|o| >= 4 under bf16) is held to that bound plus 1e-3 and reported separately."""
+    err = np.abs(o_gpu - o_ref)
+    if extra is not None:
+        allowed = bar + extra
+        big = np.zeros_like(err, dtype=bool)
+    else:
+        big = bf16_ulp_half(o_ref) > bar if bar >= 1e-3 else np.zeros_like(err, dtype=bool)
+        allowed = np.where(big, bf16_ulp_half(o_ref) + 1e-3, bar)
+    bad = err > allowed
+    assert not bad.any(), (f"max err {err.max():.3e} (bar {bar}); {int(bad.sum())} elements over; worst excess "
+                           f"{(err - allowed).max():.3e}; {int(big.sum())} large-magnitude elements held to "
+                           "their bf16 bound")
+    return float(err.max()), int(big.sum())

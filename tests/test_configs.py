@@ -1,0 +1,82 @@
+"""The five workloads at full size, CUDA path vs the fp64 oracle (needs a B200).
+
+Same launches as bench.py.  The 64k-token causal workload is checked on 256 seeded query rows
+per head (forward) and on the full backward of head 0 (query rows a block at a time, full-row
+softmax), since N x N does not fit on the host."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_68_b200 import api
+from exact_io_aware_68_b200.inputs import make_inputs, sampled_rows
+from exact_io_aware_68_b200.workloads import WORKLOADS
+from helpers import (GRAD_REL_L2, LSE_MAX_ABS, O_MAX_ABS_BF16, O_MAX_ABS_F32, assert_o_close, key_lens_device,
+                     rel_l2, run_fwd, to_device, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_fp32_head_128x64():
+    w = WORKLOADS["fp32_1x1x128x64"]
+    x = make_inputs(w, with_do=False)
+    *_, o, lse = run_fwd(x)
+    O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"])
+    err = np.abs(o.double().cpu().numpy() - O).max()
+    assert err <= O_MAX_ABS_F32, err
+    assert np.abs(lse.cpu().numpy() - L).max() <= LSE_MAX_ABS
+
+
+@pytest.mark.parametrize("name", ["bf16_4x16x1024x64", "bf16_causal_2x16x4096x128",
+                                  "bf16_keypad_dropout_16x16x512x64"])
+def test_full_workload(name):
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    q, k, v, o, lse = run_fwd(x)
+    do = to_device(x, "do")
+    dq, dk, dv = api.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, key_lens_device(x), w.dropout_p, w.seed)
+    api.check()
+    O, L = oracle.forward(x["q64"], x["k64"], x["v64"], w.scale, w.causal, x["key_lens"], w.dropout_p, w.seed)
+    o_err, n_big = assert_o_close(to_f64(o), O, O_MAX_ABS_BF16)
+    l_err = float(np.abs(lse.cpu().numpy() - L).max())
+    assert l_err <= LSE_MAX_ABS, l_err
+    ref = oracle.backward(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, w.causal, x["key_lens"], w.dropout_p,
+                          w.seed)
+    errs = {n: rel_l2(to_f64(g), r) for n, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref)}
+    print(f"{name}: O max-abs {o_err:.3e} ({n_big} elements |O|>=4), lse {l_err:.3e}, rel-L2 {errs}")
+    for n, e in errs.items():
+        assert e <= GRAD_REL_L2, (n, e)
+
+
+def test_long_context_64k():
+    w = WORKLOADS["bf16_causal_1x16x65536x64"]
+    x = make_inputs(w)
+    q, k, v, o, lse = run_fwd(x)
+    do = to_device(x, "do")
+    dq, dk, dv = api.attention_bwd(q, k, v, o, lse, do, w.scale, True)
+    api.check()
+    o64, lse_h = to_f64(o), lse.cpu().numpy()
+    worst, big = 0.0, 0
+    t0 = time.time()
+    for h in range(w.H):
+        rows = sampled_rows(w.seed, h, w.N, w.sample_rows)
+        O, L = oracle.forward_rows(x["q64"], x["k64"], x["v64"], w.scale, True, None, 0.0, w.seed, 0, h, rows)
+        e, nb = assert_o_close(o64[0, h, rows], O, O_MAX_ABS_BF16)
+        worst, big = max(worst, e), big + nb
+        assert np.abs(lse_h[0, h, rows] - L).max() <= LSE_MAX_ABS
+    t1 = time.time()
+    ref = oracle.backward_head_blocked(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, True, None, 0.0, w.seed,
+                                       0, 0, block=256)
+    errs = {n: rel_l2(to_f64(g)[0, 0], r) for n, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref)}
+    print(f"64k: forward rows max-abs {worst:.3e} ({big} elements |O|>=4) in {t1 - t0:.0f}s; head-0 backward "
+          f"rel-L2 {errs} in {time.time() - t1:.0f}s")
+    for n, e in errs.items():
+        assert e <= GRAD_REL_L2, (n, e)
+    # every head's gradients are finite; rows past the sampled ones are checked via invariants
+    for g in (dq, dk, dv):
+        assert torch.isfinite(g.float()).all()
+    # sum_j dK_j = 0 per head (the rows of dS sum to zero), a property at any size
+    s = dk.double().sum(dim=2).abs().max().item()
+    assert s <= 1e-2 * dk.double().abs().sum(dim=2).max().item()
