@@ -313,14 +313,30 @@ def run_native(args, w, world, rank, local):
     return line
 
 
+def csrc_hash():
+    """Hash of the kernel sources, to tell whether a stored ncu figure still describes them."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_68_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel, workload):
-    """dram bytes per launch of ``kernel`` from the committed ncu summary, or None."""
+    """dram bytes (read + write) per launch of ``kernel`` from the committed ncu summary; None when
+    there is none or the kernel sources changed since it was captured."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    return d.get(workload, {}).get(kernel)
+    e = d.get(workload, {}).get(kernel)
+    if e is None or e.get("csrc_hash") != csrc_hash():
+        return None
+    return e["dram_bytes"]
 
 
 # ----------------------------------------------------------------------------- oracle timing
