@@ -23,6 +23,8 @@ SIGNATURES = {
     "fa_bwd_prep": (_I, [_P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "fa_bwd_main": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P, _SZ, _P]),
     "fa_bwd_dq_convert": (_I, [_P, _I, _I, _I, _I, _F, _P, _SZ, _P]),
+    "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P]),
+    "fa_bwd_noalloc_max_scratch": (_SZ, []),
     "fa_dropout_mask": (_I, [_P, _I, _I, _I, _F, _U64, _P]),
     "fa_check": (_I, [_P]),
     "fa_get_error": (ctypes.c_char_p, []),

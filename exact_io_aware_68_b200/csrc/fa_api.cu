@@ -364,3 +364,63 @@ void fa_debug_set_flags(int flags) { g_debug_flags.store(flags); }
 const char* fa_version(void) { return "exact-io-aware-attention sm_100a 0.1"; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------- backward without allocation
+// Some callers cannot allocate device memory: a plugin running inside another runtime that owns
+// every byte of device memory and gives its plugins no workspace, or a latency-critical loop where
+// the implicit device synchronisation of cudaMalloc is not acceptable.  fa_bwd_noalloc serves
+// them: the backward's scratch (the fp32 dQ accumulator and D) lives in the fixed array below,
+// which is part of the library image.  Every GPU that loads the library holds these bytes until
+// the process exits.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(48) << 20;   // 48 MiB
+static __device__ __align__(256) unsigned char g_fa_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// The device address of the scratch array on the current device.  In host code the array's name
+// is only a host-side stand-in, so the address is looked up once per device (with that device
+// current) and cached.
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device ordinal %d is out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fa_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(FA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                         void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                         const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream) {
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need > kNoallocScratchBytes)
+    return fail(FA_ERR_INVALID_ARG,
+                "fa_bwd_noalloc: B=%d H=%d N=%d d=%d needs %zu bytes of scratch, more than the library's "
+                "static %zu bytes; call fa_bwd with a workspace instead",
+                B, H, N, d, need, kNoallocScratchBytes);
+  void* ws = nullptr;
+  const fa_status st = noalloc_scratch(&ws);
+  if (st != FA_OK) return st;
+  return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, key_lens, dropout_p, seed, ws,
+                kNoallocScratchBytes, stream);
+}
+
+size_t fa_bwd_noalloc_max_scratch(void) { return kNoallocScratchBytes; }
+
+}  // extern "C"

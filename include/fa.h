@@ -99,6 +99,26 @@ FA_API fa_status fa_bwd_main(const void* q, const void* k, const void* v, const 
 FA_API fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward that allocates nothing, for callers that cannot allocate device memory: a plugin
+ * inside another runtime that owns all device memory and hands it no workspace, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit device synchronisation.
+ * (The paper has no counterpart: this is an interface convenience of this library.)
+ * Same arguments and results as fa_bwd, minus the workspace: the scratch (fp32 dQ accumulator
+ * and D, fa_bwd_workspace_size() bytes) lives in a fixed 48 MiB array inside the library, which
+ * every GPU that loads the library keeps until the process exits.  Sizes whose scratch exceeds
+ * fa_bwd_noalloc_max_scratch() are rejected with FA_ERR_INVALID_ARG.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device current; make
+ * that first call before any stream capture.  All calls share the one array: calls that may
+ * overlap on the GPU (other streams, other threads) race and give wrong gradients; serialise
+ * them.  Each call clears the part of the array that must start at zero. */
+FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv,
+                         int B, int H, int N, int d, float scale, int causal,
+                         const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream);
+
+/* Size in bytes of fa_bwd_noalloc's static scratch array (48 MiB). */
+FA_API size_t fa_bwd_noalloc_max_scratch(void);
+
 /* Writes the dropout keep decisions (1 = kept, 0 = dropped) of every element into
  * keep (uint8 [B,H,N,N], device).  For testing the counter hash bit for bit. */
 FA_API fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, uint64_t seed,
