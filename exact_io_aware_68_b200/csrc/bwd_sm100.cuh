@@ -129,7 +129,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
 }
 
-template <int D>
+template <int D, bool DROPOUT>
 __global__ void __launch_bounds__(320, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -362,7 +362,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int e = 0; e < 16; ++e) {
           const int c = ch * 32 + 2 * e;
           float a = pr[c], bb = pr[c + 1];
-          if (p.dropout) {
+          if (DROPOUT) {
             // element (query i = qrow0 + c, key j = key): ctr = (bh*N + i)*N + j
             const uint64_t ctr = drop_col0 + uint64_t(c) * uint64_t(p.N);
             const bool ka = dropout_keep(p.seed, ctr, p.drop_thr);
@@ -398,7 +398,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int e = 0; e < 16; ++e) {
           const int c = ch * 32 + 2 * e;
           float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
-          if (p.dropout) {
+          if (DROPOUT) {
             dpa = ((keep_bits[ch] >> (2 * e)) & 1u) ? dpa * p.drop_scale : 0.f;
             dpb = ((keep_bits[ch] >> (2 * e + 1)) & 1u) ? dpb * p.drop_scale : 0.f;
           }
@@ -431,7 +431,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
     } else if (ok && warp_wait(fin, 0, wc)) {
       tc_fence_after();
-      const float s = p.dropout ? p.drop_scale : 1.f;
+      const float s = DROPOUT ? p.drop_scale : 1.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t vr[32];

@@ -127,25 +127,25 @@ fa_status set_smem(K kernel, int bytes) {
   return FA_OK;
 }
 
-template <int D>
+template <int D, bool DROPOUT>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::FwdParams& p,
                      cudaStream_t s) {
   using L = fa::FwdLayout<D>;
-  fa_status st = set_smem(fa::fa_fwd_sm100_kernel<D>, L::BYTES);
+  fa_status st = set_smem(fa::fa_fwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
   const dim3 grid(p.n_qtiles, p.B * p.H);
-  fa::fa_fwd_sm100_kernel<D><<<grid, 192, L::BYTES, s>>>(mq, mk, mv, p);
+  fa::fa_fwd_sm100_kernel<D, DROPOUT><<<grid, 192, L::BYTES, s>>>(mq, mk, mv, p);
   return launch_status("fa_fwd kernel launch");
 }
 
-template <int D>
+template <int D, bool DROPOUT>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                           const fa::BwdParams& p, cudaStream_t s) {
   using L = fa::BwdLayout<D>;
-  fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D>, L::BYTES);
+  fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
   const dim3 grid(p.n_tiles, p.B * p.H);
-  fa::fa_bwd_sm100_kernel<D><<<grid, 320, L::BYTES, s>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, 320, L::BYTES, s>>>(mq, mk, mv, mdo, p);
   return launch_status("fa_bwd main kernel launch");
 }
 
@@ -210,7 +210,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.wait_ns = g_wait_ns.load();
   p.debug_flags = g_debug_flags.load();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_fwd<64>(mq, mk, mv, p, s) : launch_fwd<128>(mq, mk, mv, p, s);
+  if (d == 64) return p.dropout ? launch_fwd<64, true>(mq, mk, mv, p, s) : launch_fwd<64, false>(mq, mk, mv, p, s);
+  return p.dropout ? launch_fwd<128, true>(mq, mk, mv, p, s) : launch_fwd<128, false>(mq, mk, mv, p, s);
 }
 
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
@@ -296,7 +297,10 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* 
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd_main<64>(mq, mk, mv, mdo, p, s) : launch_bwd_main<128>(mq, mk, mv, mdo, p, s);
+  if (d == 64)
+    return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, s) : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, s);
+  return p.dropout ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, s)
+                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, s);
 }
 
 fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,

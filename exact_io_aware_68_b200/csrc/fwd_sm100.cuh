@@ -57,7 +57,7 @@ struct FwdLayout {
   static_assert(BYTES <= 232448, "shared memory budget");
 };
 
-template <int D>
+template <int D, bool DROPOUT>
 __global__ void __launch_bounds__(192, 1)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -227,18 +227,15 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (lane == 0) mbar_arrive(&s_empty[sb]);
 
       const int k0 = j * 128;
-      const bool need_mask = (k0 + 128 > kv_end) || (p.causal && k0 + 128 > q0);
+      if ((k0 + 128 > kv_end) || (p.causal && k0 + 128 > q0)) {   // block straddles a mask edge
+        const int lim = min(kv_end, p.causal ? q_row + 1 : kv_end) - k0;   // columns < lim are kept
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float x = __uint_as_float(sr[c]);
-        if (need_mask) {
-          const int col = k0 + c;
-          if (col >= kv_end || (p.causal && col > q_row)) x = -INFINITY;
-        }
-        sr[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
-      }
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
       const float m_cand = mx * sl2;
       float alpha = 1.f;
       if (m_cand > m_ref + kRescaleThreshold) {
@@ -253,7 +250,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_use));
         float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_use));
         rs += p0 + p1;
-        if (p.dropout) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
+        if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
           const uint64_t ctr = drop_row + uint64_t(k0 + 2 * c);
           p0 = dropout_keep(p.seed, ctr, p.drop_thr) ? p0 : 0.f;
           p1 = dropout_keep(p.seed, ctr + 1, p.drop_thr) ? p1 : 0.f;
@@ -301,7 +298,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
     } else if (ok && mbar_wait(o_done, (n_kv - 1) & 1, wc)) {
       tc_fence_after();
-      const float inv_l = l > 0.f ? (p.dropout ? p.drop_scale : 1.f) / l : 0.f;
+      const float inv_l = l > 0.f ? (DROPOUT ? p.drop_scale : 1.f) / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];

@@ -22,11 +22,6 @@ __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_fa_device
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 __device__ __forceinline__ float ex2_approx(float x) {   // MUFU 2^x
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -79,31 +74,45 @@ struct WaitCtl {
   volatile int* abort;   // shared memory
 };
 
+// SM cycles that cover `ns` nanoseconds at any SM clock up to 2 GHz (a lower clock only makes
+// the bound longer in wall time, never shorter).
+__device__ __forceinline__ long long wait_cycles(uint64_t ns) { return (long long)(ns * 2ull); }
+
 // Wait until the phase with parity `parity` of `bar` has completed.  Returns false (after
 // recording kStatusTimeout and raising the abort flag) when the limit runs out, or when
-// another role of the CTA has already raised the abort flag.
+// another role of the CTA has already raised the abort flag.  The fast path is one try_wait;
+// the slow path reads the SM's own cycle counter (cheap, unlike %globaltimer) and the abort flag
+// only every 32 unsuccessful polls, so completion is noticed without added latency.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   const uint32_t a = smem_u32(bar);
   if (mbar_test(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  const long long t0 = clock64();
+  const long long limit = wait_cycles(w.limit_ns);
+  for (uint32_t it = 1;; ++it) {
     if (mbar_test(a, parity)) return true;
-    if (*w.abort) return false;
-    if (globaltimer_ns() - t0 > w.limit_ns) {
-      record_status(kStatusTimeout);
-      *w.abort = 1;
-      return false;
+    if ((it & 31u) == 0) {
+      if (*w.abort) return false;
+      if (clock64() - t0 > limit) {
+        record_status(kStatusTimeout);
+        *w.abort = 1;
+        return false;
+      }
     }
   }
 }
 // Same, but ignores the abort flag: used while unwinding, to drain work already in flight.
 __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_test(a, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) { record_status(kStatusTimeout); return false; }
+  if (mbar_test(a, parity)) return true;
+  const long long t0 = clock64();
+  const long long limit = wait_cycles(limit_ns);
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(a, parity)) return true;
+    if ((it & 31u) == 0 && clock64() - t0 > limit) {
+      record_status(kStatusTimeout);
+      return false;
+    }
   }
-  return true;
 }
 
 // ----------------------------------------------------------------------------- TMA
