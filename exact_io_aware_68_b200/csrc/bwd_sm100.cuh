@@ -14,16 +14,20 @@
 //                         mixed-precision advice in section 3.2 of the same blog post asks)
 //   fa_bwd_dq_kernel      dQ = bf16(tau * accumulator)
 //
-// Main kernel roles (10 warps):
-//   warps 0-3  compute: thread r owns key row r (TMEM lane r): P^T = exp2(S^T*tau*log2e - lse2),
-//              masks, dropout, writes (P*Z)^T (bf16) to TMEM (dV takes 1/(1-p) at the end); dS^T = P^T * (dP^T - D) to TMEM (bf16)
-//              and dS to shared memory (MN-major, the A operand of dQ = dS K); dV epilogue
-//   warps 4-7  dQ: read the 128 x D dQ tile from TMEM, atomically add to the accumulator; dK epilogue
+// Main kernel roles (12 warps, three warpgroups with their own register budgets):
+//   warps 0-3  compute (248 registers): thread r owns key row r (TMEM lane r).
+//              P^T = exp2(S^T tau log2e - lse2), masks, dropout; (P*Z)^T as bf16 into TMEM (dV
+//              takes 1/(1-p) at the end); dS^T = P^T (dP^T Z/(1-p) - D) as bf16 into TMEM (for dK)
+//              and into shared memory (one tile read by the dQ MMA as an MN-major operand); dV epilogue
+//   warps 4-7  dQ (168 registers): read the dQ^T tile from TMEM (lane = feature, column = query),
+//              stage it in shared memory (the dS buffer, free once the dQ MMA is done) and add it to
+//              the fp32 accumulator with TMA bulk reductions, one per warp; dK epilogue
 //   warp 8     producer: TMA K, V once; Q, dO per query tile (STAGES deep); lse and D per tile
-//   warp 9     MMA issuer
-// TMEM (512 columns): ST [0,128) S^T then P~^T in [0,64); DPT [128,256) dP^T then dS^T in
-// [128,192); dV [256,256+D); dK [256+D,256+2D).  dQ: D=64 -> [384,448); D=128 -> the upper
-// halves [64,128) and [192,256), so the next S^T / dP^T waits until dQ has been read.
+//   warp 9     MMA issuer; warps 10-11 idle (88 registers for warps 8-11)
+// TMEM (512 columns): ST [0,128) S^T then (P*Z)^T in [0,64); DPT [128,256) dP^T then dS^T in
+// [128,192); dV [256,256+D); dK [256+D,256+2D).  dQ^T = K^T dS^T: D=64 -> M=64, N=128 in
+// [384,512); D=128 -> two N=64 halves in [64,128) and [192,256), so the next S^T / dP^T waits
+// until dQ^T has been read.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -31,7 +35,7 @@
 
 namespace fa {
 
-struct BwdParams {
+struct BwdParams {  // (the main kernel also takes tensor maps of q, k, v, dO and the dQ accumulator)
   const __nv_bfloat16* o;      // [B,H,N,D]   (prep)
   const __nv_bfloat16* dO;     // [B,H,N,D]   (prep)
   const float* lse;            // [B,H,N]
@@ -115,12 +119,18 @@ struct BwdLayout {
   static constexpr int STAT_OFF = DS_OFF + 2 * SUB;           // per stage: lse2[128], D[128]
   static constexpr int BAR_OFF = STAT_OFF + STAGES * 1024;
   // kv_full, q_full[S], do_full[S], stat_full[S], q_empty[S], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_empty, fin
-  static constexpr int NBARS = 1 + 4 * STAGES + 7;
+  // dq_full, dq_empty, ds_free, fin
+  static constexpr int NBARS = 1 + 4 * STAGES + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ST_COL = 0, DPT_COL = 128, DV_COL = 256, DK_COL = 256 + D;
   static constexpr int TMEM_COLS = 512;
+  // dQ staging (in the dS buffer): per warp and round, QPR queries x FPW features of fp32
+  static constexpr int FPW = (D == 128) ? 32 : 16;     // features per warp (TMEM lanes with data)
+  static constexpr int QPR = (D == 128) ? 64 : 128;    // queries per reduction round
+  static constexpr int ROUNDS = 128 / QPR;
+  static constexpr int STAGE_BYTES = QPR * FPW * 4;    // 8 KB per warp
+  static_assert(4 * STAGE_BYTES <= 2 * SUB, "dQ staging fits in the dS buffer");
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
@@ -129,11 +139,20 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
 }
 
+// Bulk tensor reduction (add) of a shared-memory box into global memory; no multicast.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int D, bool DROPOUT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
   constexpr int STAGES = L::STAGES;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -154,7 +173,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* ds_full = p_full + 1;
   uint64_t* dq_full = ds_full + 1;
   uint64_t* dq_empty = dq_full + 1;
-  uint64_t* fin = dq_empty + 1;
+  uint64_t* ds_free = dq_empty + 1;
+  uint64_t* fin = ds_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
@@ -183,6 +203,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(ds_full, 4);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 4);
+    mbar_init(ds_free, 4);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -199,8 +220,13 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const WaitCtl wc{p.wait_ns, abort_flag};
   const uint64_t row_base = uint64_t(bh) * uint64_t(p.N);
 
-  if (warp == 8) {
+  // Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
+  // 128 x (248 + 168 + 88) = 64512.  Each role lowers or raises its budget first thing.
+  if (warp >= 10) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+  } else if (warp == 8) {
     // =========================================================== producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
     int issued = 0;
     if (n_iter > 0) {
       if (lane == 0) {
@@ -208,6 +234,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
         prefetch_tmap(&tm_do);
+        prefetch_tmap(&tm_dq);
         mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -257,10 +284,11 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp == 9) {
     // =========================================================== MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
     if (lane == 0 && n_iter > 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (or V) K-major, Q (or dO) K-major
-      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // A in TMEM, B MN-major
-      constexpr uint32_t kIdQ = idesc_bf16(128, 64, true, true);      // dS MN-major, K MN-major, N = 64
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);             // K (V) and Q (dO) K-major
+      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);                // A in TMEM, B MN-major
+      constexpr uint32_t kIdQ = idesc_bf16(D, D == 128 ? 64 : 128, true, true);  // K^T, dS^T: both MN-major
       const uint32_t k_base = smem_u32(smem + L::K_OFF);
       const uint32_t v_base = smem_u32(smem + L::V_OFF);
       const uint32_t ds_base = smem_u32(smem + L::DS_OFF);
@@ -291,7 +319,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                  kIdS, kk > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
-        // dV += P~^T dO   (A = P~^T in TMEM, B = dO MN-major: N = D, K = queries)
+        // dV += (P*Z)^T dO   (A = (P*Z)^T in TMEM, B = dO MN-major: N = D, K = queries)
         if (!mbar_wait(p_full, t & 1, wc)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -305,15 +333,21 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + L::DK_COL, tmem + L::DPT_COL + kk * 8, sdesc_sw128(q_base + kk * 2048, L::SUB, 1024), kIdG,
                  (t > 0 || kk > 0) ? 1u : 0u);
-        // dQ_tile = dS K   (M = 128 queries, K = 128 keys, N = 64 per panel of D)
+        // dQ^T tile = K^T dS^T   (M = D features, K = 128 keys, N = queries)
         if (D == 64 && t >= 1 && !mbar_wait(dq_empty, (t - 1) & 1, wc)) { ok = false; break; }
+        if (D == 128) {
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-          const uint32_t dq_col = (D == 64) ? 384u : (h == 0 ? 64u : 192u);
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + (h == 0 ? 64u : 192u), sdesc_sw128(k_base + kk * 2048, L::SUB, 1024),
+                     sdesc_sw128(ds_base + h * L::SUB + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
+          }
+        } else {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + dq_col, sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024),
-                   sdesc_sw128(k_base + h * L::SUB + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + 384u, sdesc_sw128(k_base + kk * 2048, L::SUB, 1024),
+                   sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
         }
         mma_commit(dq_full);
         mma_commit(&q_empty[st]);
@@ -324,6 +358,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp < 4) {
     // =========================================================== compute (key row r)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 248;\n" ::: "memory");
     const int r = tid;
     const int key = k0 + r;
     const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
@@ -338,82 +373,88 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (!warp_wait(s_full, t & 1, wc)) { ok = false; break; }
       if (!warp_wait(&stat_full[st], (t / STAGES) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      float pr[128];                 // P^T row (undropped), fp32
-      uint32_t keep_bits[4] = {0u, 0u, 0u, 0u};
-      const uint64_t drop_col0 = (row_base + uint64_t(qrow0)) * uint64_t(p.N) + uint64_t(key);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sr[32];
-        tmem_ld32(lane_base + L::ST_COL + ch * 32, sr);
+      // ---- P^T = exp2(S^T tau log2e - lse2): one pass over the 128 query columns
+      float pr[128];
+      {
+        uint32_t* sr = reinterpret_cast<uint32_t*>(pr);
+        tmem_ld32(lane_base + L::ST_COL + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(lane_base + L::ST_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(lane_base + L::ST_COL + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(lane_base + L::ST_COL + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
         tmem_ld_wait();
-        reg_fence32(sr);
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = ch * 32 + e;
-          float pv = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -st_l[c]));
-          if (need_mask) {
-            const int q = qrow0 + c;
-            if (key >= kv_end || q >= p.N || (p.causal && key > q)) pv = 0.f;
-          }
-          pr[c] = pv;
-        }
+        for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
+      }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = ch * 32 + 2 * e;
-          float a = pr[c], bb = pr[c + 1];
+      for (int c = 0; c < 128; ++c) pr[c] = ex2_approx(fmaf(pr[c], sl2, -st_l[c]));
+      if (need_mask) {
+        // allowed: key < kv_end, query < N, and (not causal or key <= query)
+        const int lim_q = p.N - qrow0;                                  // query columns < lim_q exist
+        const int from_q = p.causal ? key - qrow0 : -1;                 // causal: columns >= from_q
+        const bool key_ok = key < kv_end;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (!key_ok || c >= lim_q || c < from_q) pr[c] = 0.f;
+      }
+      uint32_t keep_bits[4] = {0u, 0u, 0u, 0u};
+      {
+        const uint64_t drop_col0 = (row_base + uint64_t(qrow0)) * uint64_t(p.N) + uint64_t(key);
+        uint32_t pk[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          float a = pr[2 * e], bb = pr[2 * e + 1];
           if (DROPOUT) {
             // element (query i = qrow0 + c, key j = key): ctr = (bh*N + i)*N + j
-            const uint64_t ctr = drop_col0 + uint64_t(c) * uint64_t(p.N);
+            const uint64_t ctr = drop_col0 + uint64_t(2 * e) * uint64_t(p.N);
             const bool ka = dropout_keep(p.seed, ctr, p.drop_thr);
             const bool kb = dropout_keep(p.seed, ctr + uint64_t(p.N), p.drop_thr);
-            keep_bits[ch] |= (ka ? 1u : 0u) << (2 * e);
-            keep_bits[ch] |= (kb ? 1u : 0u) << (2 * e + 1);
+            keep_bits[e >> 4] |= (ka ? 1u : 0u) << (2 * (e & 15));
+            keep_bits[e >> 4] |= (kb ? 1u : 0u) << (2 * (e & 15) + 1);
             a = ka ? a : 0.f;      // P * Z; dV takes the 1/(1-p) factor in its fp32 epilogue
             bb = kb ? bb : 0.f;
           }
           pk[e] = pack_bf16x2(a, bb);
         }
-        // P~^T columns [16ch, 16ch+16) overlay score columns already read
-        tmem_st16(lane_base + L::ST_COL + ch * 16, pk);
+        // (P*Z)^T overlays the first 64 score columns, already read
+        tmem_st32(lane_base + L::ST_COL + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(lane_base + L::ST_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
 
-      // ---- dS^T = P^T * (dP^T - D)
+      // ---- dS^T = P^T * (dP^T Z/(1-p) - D), two halves of 64 query columns
       if (!warp_wait(dp_full, t & 1, wc)) { ok = false; break; }
-      // the previous dQ MMA has finished reading the dS tile in shared memory
-      if (t >= 1 && !warp_wait(dq_full, (t - 1) & 1, wc)) { ok = false; break; }
+      // the dQ warps have finished with the shared dS buffer (the last dQ MMA and its reductions)
+      if (t >= 1 && !warp_wait(ds_free, (t - 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t dr[32];
-        tmem_ld32(lane_base + L::DPT_COL + ch * 32, dr);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t dr[64];
+        tmem_ld32(lane_base + L::DPT_COL + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+        tmem_ld32(lane_base + L::DPT_COL + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
         tmem_ld_wait();
-        reg_fence32(dr);
-        uint32_t pk[16];
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = ch * 32 + 2 * e;
+        for (int e = 0; e < 32; ++e) {
+          const int c = 64 * hh + 2 * e;
           float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
           if (DROPOUT) {
-            dpa = ((keep_bits[ch] >> (2 * e)) & 1u) ? dpa * p.drop_scale : 0.f;
-            dpb = ((keep_bits[ch] >> (2 * e + 1)) & 1u) ? dpb * p.drop_scale : 0.f;
+            const uint32_t kbits = keep_bits[c >> 5];
+            dpa = ((kbits >> (c & 31)) & 1u) ? dpa * p.drop_scale : 0.f;
+            dpb = ((kbits >> ((c + 1) & 31)) & 1u) ? dpb * p.drop_scale : 0.f;
           }
-          const float dsa = pr[c] * (dpa - st_l[128 + c]);
-          const float dsb = pr[c + 1] * (dpb - st_l[128 + c + 1]);
-          pk[e] = pack_bf16x2(dsa, dsb);
+          pk[e] = pack_bf16x2(pr[c] * (dpa - st_l[128 + c]), pr[c + 1] * (dpb - st_l[128 + c + 1]));
         }
-        tmem_st16(lane_base + L::DPT_COL + ch * 16, pk);
-        // dS (queries contiguous) into the 128-byte-swizzled panel: row = key r, 16-byte chunks
-        const int panel = ch >> 1;
+        tmem_st32(lane_base + L::DPT_COL + 32 * hh, pk);
+        // dS (queries contiguous) into the 128-byte-swizzled panel hh: row = key r, 16-byte chunks
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
-          const int chunk = (ch & 1) * 4 + v4;   // 8 queries per 16-byte chunk
-          uint4* dst = reinterpret_cast<uint4*>(ds_smem + panel * L::SUB + r * 128 + ((chunk ^ (r & 7)) << 4));
-          *dst = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        for (int chunk = 0; chunk < 8; ++chunk) {   // 8 queries per 16-byte chunk
+          uint4* dst = reinterpret_cast<uint4*>(ds_smem + hh * L::SUB + r * 128 + ((chunk ^ (r & 7)) << 4));
+          *dst = make_uint4(pk[4 * chunk], pk[4 * chunk + 1], pk[4 * chunk + 2], pk[4 * chunk + 3]);
         }
       }
       fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
@@ -450,36 +491,61 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
     }
   } else {
-    // =========================================================== dQ readout + dK epilogue (warps 4-7)
+    // =========================================================== dQ + dK epilogue (warps 4-7)
+    // TMEM holds dQ^T: lane = feature, column = query.  D=128: feature 32*quarter + lane;
+    // D=64 (M=64 layout): feature 16*quarter + lane on lanes 0-15.  Each warp stages its
+    // features for QPR queries in its 8 KB slice of the dS buffer ([query][feature], fp32) and
+    // adds that box to the accumulator with one TMA bulk reduction.
     const int quarter = warp - 4;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    float* stage = reinterpret_cast<float*>(smem + L::DS_OFF + quarter * L::STAGE_BYTES);
+    const bool lane_ok = lane < L::FPW;
     bool ok = true;
     for (int t = 0; t < n_iter; ++t) {
-      const int q = (q_first + t) * 128 + r;
+      const int qrow0 = (q_first + t) * 128;
       if (!warp_wait(dq_full, t & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      uint32_t g[D];
+      uint32_t g[128];
+      if (D == 128) {
+        tmem_ld32(lane_base + 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
+        tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
+        tmem_ld32(lane_base + 192, *reinterpret_cast<uint32_t(*)[32]>(&g[64]));
+        tmem_ld32(lane_base + 224, *reinterpret_cast<uint32_t(*)[32]>(&g[96]));
+      } else {
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        const uint32_t col = (D == 64) ? 384u : (h == 0 ? 64u : 192u);
-        tmem_ld32(lane_base + col, *reinterpret_cast<uint32_t(*)[32]>(&g[h * 64]));
-        tmem_ld32(lane_base + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&g[h * 64 + 32]));
+        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + 384 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&g[32 * c]));
       }
       tmem_ld_wait();
 #pragma unroll
-      for (int h = 0; h < D / 32; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&g[h * 32]));
+      for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&g[h * 32]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_empty);
-      if (q < p.N) {
-        float4* dst = reinterpret_cast<float4*>(p.dq_acc + (row_base + q) * D);
+      // the dQ MMA has completed, so the dS buffer is free for staging
 #pragma unroll
-        for (int c = 0; c < D / 4; ++c)
-          atomicAdd(dst + c, make_float4(__uint_as_float(g[4 * c]), __uint_as_float(g[4 * c + 1]),
-                                         __uint_as_float(g[4 * c + 2]), __uint_as_float(g[4 * c + 3])));
+      for (int rd = 0; rd < L::ROUNDS; ++rd) {
+        if (rd > 0) {   // the previous round's reduction must have read the staging slice
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+        }
+        if (lane_ok) {
+#pragma unroll
+          for (int c = 0; c < L::QPR; ++c) stage[c * L::FPW + lane] = __uint_as_float(g[rd * L::QPR + c]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, stage, quarter * L::FPW, qrow0 + rd * L::QPR, bh);
+          bulk_commit();
+        }
       }
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_free);
     }
+    if (lane == 0) bulk_wait0();   // every reduction has completed before the kernel ends
+    __syncwarp();
     const int key = k0 + r;
     if (n_iter == 0) {
       if (key < p.N) {

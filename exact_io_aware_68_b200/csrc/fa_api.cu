@@ -70,6 +70,22 @@ fa_status make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int d,
   return FA_OK;
 }
 
+// 3-D view {d, N, B*H} of the fp32 dQ accumulator for the backward's TMA bulk reductions:
+// boxes of (features per warp) x (queries per round), no swizzle; rows past N are not written.
+fa_status make_dq_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  const cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
+  const cuuint32_t box[3] = {d == 128 ? 32u : 16u, d == 128 ? 64u : 128u, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled(dQ accumulator) failed with CUresult %d", int(r));
+  return FA_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 fa_status check_common(int B, int H, int N, int d, float scale, float dropout_p, bool bf16) {
@@ -140,12 +156,12 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 template <int D, bool DROPOUT>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                          const fa::BwdParams& p, cudaStream_t s) {
+                          const CUtensorMap& mdq, const fa::BwdParams& p, cudaStream_t s) {
   using L = fa::BwdLayout<D>;
   fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
   const dim3 grid(p.n_tiles, p.B * p.H);
-  fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, 320, L::BYTES, s>>>(mq, mk, mv, mdo, p);
+  fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, 384, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status("fa_bwd main kernel launch");
 }
 
@@ -287,20 +303,22 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* 
   FA_CHECK_PTR(dv);
   Workspace w;
   if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if ((st = make_tile_map(&mq, q, B * H, N, d, "q")) != FA_OK) return st;
   if ((st = make_tile_map(&mk, k, B * H, N, d, "k")) != FA_OK) return st;
   if ((st = make_tile_map(&mv, v, B * H, N, d, "v")) != FA_OK) return st;
   if ((st = make_tile_map(&mdo, dO, B * H, N, d, "dO")) != FA_OK) return st;
+  if ((st = make_dq_map(&mdq, w.dq_acc, B * H, N, d)) != FA_OK) return st;
   fa::BwdParams p = bwd_params(B, H, N, scale, causal, key_lens, dropout_p, seed, w);
   p.lse = lse;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, s) : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, s);
-  return p.dropout ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, s)
-                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, s);
+    return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, p, s)
+                     : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, p, s);
+  return p.dropout ? launch_bwd_main<128, true>(mq, mk, mv, mdo, mdq, p, s)
+                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, mdq, p, s);
 }
 
 fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
