@@ -16,7 +16,7 @@
 //
 // Main kernel roles (12 warps, three warpgroups with their own register budgets):
 //   warps 0-3  compute (248 registers): thread r owns key row r (TMEM lane r).
-//              P^T = exp2(S^T tau log2e - lse2), masks, dropout; (P*Z)^T as bf16 into TMEM (dV
+//              P^T = exp2(S^T tau log2e - lse2) (packed f32x2 arithmetic), masks, dropout; (P*Z)^T as bf16 into TMEM (dV
 //              takes 1/(1-p) at the end); dS^T = P^T (dP^T Z/(1-p) - D) as bf16 into TMEM (for dK)
 //              and into shared memory (one tile read by the dQ MMA as an MN-major operand); dV epilogue
 //   warps 4-7  dQ (168 registers): read the dQ^T tile from TMEM (lane = feature, column = query),
@@ -256,7 +256,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(smem + L::DO_OFF + st * L::TILE + c * L::SUB, &tm_do, &do_full[st], c * 64, qrow0, bh);
         }
-        // per-query statistics of this tile: lse in the exp2 domain and D
+        // per-query statistics of this tile, negated: -lse in the exp2 domain and -D
         float* st_l = stat + st * 256;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -264,8 +264,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const int q = qrow0 + c;
           float lv = 0.f, dv = 0.f;
           if (q < p.N) {
-            lv = p.lse[row_base + q] * kLog2e;
-            dv = p.dvec[row_base + q];
+            lv = -p.lse[row_base + q] * kLog2e;
+            dv = -p.dvec[row_base + q];
           }
           st_l[c] = lv;
           st_l[128 + c] = dv;
@@ -326,15 +326,11 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_sw128(do_base + kk * 2048, L::SUB, 1024), kIdG,
                  (t > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q
+        // dQ^T tile = K^T dS^T   (M = D features, K = 128 keys, N = queries), issued before dK so
+        // that the dQ warps read it out while dK runs
         if (!mbar_wait(ds_full, t & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::DK_COL, tmem + L::DPT_COL + kk * 8, sdesc_sw128(q_base + kk * 2048, L::SUB, 1024), kIdG,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        // dQ^T tile = K^T dS^T   (M = D features, K = 128 keys, N = queries)
         if (D == 64 && t >= 1 && !mbar_wait(dq_empty, (t - 1) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
         if (D == 128) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -350,6 +346,11 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                    sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
         }
         mma_commit(dq_full);
+        // dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::DK_COL, tmem + L::DPT_COL + kk * 8, sdesc_sw128(q_base + kk * 2048, L::SUB, 1024), kIdG,
+                 (t > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&q_empty[st]);
       }
       mma_commit(fin);
@@ -385,8 +386,17 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
       }
+      {
+        const uint64_t sl2x2 = f2_make(sl2, sl2);
+        const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(st_l);   // pairs of -lse2
 #pragma unroll
-      for (int c = 0; c < 128; ++c) pr[c] = ex2_approx(fmaf(pr[c], sl2, -st_l[c]));
+        for (int c = 0; c < 128; c += 2) {
+          float x0, x1;
+          f2_split(f2_fma(f2_make(pr[c], pr[c + 1]), sl2x2, nl2[c >> 1]), x0, x1);
+          pr[c] = ex2_approx(x0);
+          pr[c + 1] = ex2_approx(x1);
+        }
+      }
       if (need_mask) {
         // allowed: key < kv_end, query < N, and (not causal or key <= query)
         const int lim_q = p.N - qrow0;                                  // query columns < lim_q exist
@@ -438,6 +448,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
         reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
         uint32_t pk[32];
+        const uint64_t* nd2 = reinterpret_cast<const uint64_t*>(st_l + 128);   // pairs of -D
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = 64 * hh + 2 * e;
@@ -447,7 +458,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             dpa = ((kbits >> (c & 31)) & 1u) ? dpa * p.drop_scale : 0.f;
             dpb = ((kbits >> ((c + 1) & 31)) & 1u) ? dpb * p.drop_scale : 0.f;
           }
-          pk[e] = pack_bf16x2(pr[c] * (dpa - st_l[128 + c]), pr[c + 1] * (dpb - st_l[128 + c + 1]));
+          float da, db;   // dS = P (dP - D), as P * (dP + (-D)) on pairs
+          f2_split(f2_mul(f2_make(pr[c], pr[c + 1]), f2_add(f2_make(dpa, dpb), nd2[c >> 1])), da, db);
+          pk[e] = pack_bf16x2(da, db);
         }
         tmem_st32(lane_base + L::DPT_COL + 32 * hh, pk);
         // dS (queries contiguous) into the 128-byte-swizzled panel hh: row = key r, 16-byte chunks

@@ -149,8 +149,8 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   using L = fa::FwdLayout<D>;
   fa_status st = set_smem(fa::fa_fwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
-  const dim3 grid(p.n_qtiles, p.B * p.H);
-  fa::fa_fwd_sm100_kernel<D, DROPOUT><<<grid, 192, L::BYTES, s>>>(mq, mk, mv, p);
+  const dim3 grid((p.n_qtiles + 1) / 2, p.B * p.H);   // one CTA per pair of 128-row query tiles
+  fa::fa_fwd_sm100_kernel<D, DROPOUT><<<grid, 384, L::BYTES, s>>>(mq, mk, mv, p);
   return launch_status("fa_fwd kernel launch");
 }
 

@@ -3,12 +3,22 @@
 // "Tiling и online softmax": m <- max(m, m_block), l and O re-expressed against the new m), so
 // the N x N score matrix never reaches HBM.
 //
-// One CTA computes one work item (b, h, 128-row query tile) and loops over 128-key blocks.
-//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r); masks, exponentiates,
-//              writes P (bf16) to TMEM, rescales O when needed, writes O and lse at the end
-//   warp 4     producer: TMA loads of the Q tile and the K/V ring (STAGES deep)
-//   warp 5     MMA issuer: S = Q K^T into one of two TMEM score buffers, O += P V
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0, P1 (64 columns of packed bf16 each).
+// One CTA computes two adjacent 128-row query tiles A and B of one (b, h) and loops over 128-key
+// blocks; both tiles share every K/V block.  Warp roles (three warpgroups):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns query row r of its
+//              tile (= TMEM lane r); masks, exponentiates, writes P (bf16) over the tile's score
+//              columns, rescales O when needed, writes O and lse at the end
+//   warp 8     producer of both Q tiles and the K ring; warp 10 producer of the V ring
+//   warp 9     MMA issuer, in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while one tile's
+//              softmax runs, the tensor core works on the other tile.  P is handed over in two
+//              halves of 64 keys, so the first half of PV runs while the second half of P is made.
+//   warp 11    idle
+// Softmax arithmetic: the scale-and-shift and the row sum use packed f32x2 operations and the row
+// max a tree of three-input maxima; every exponential goes to the MUFU unit (moving a share to a
+// polynomial on the FMA pipe was measured slower: the softmax is bound by instruction issue).
+// TMEM columns: S_A [0,128), S_B [128,256) (P over the first 64 columns of each), O_A [256,256+D),
+// O_B [256+D,256+2D).  tcgen05 operations from one thread complete in issue order, so S_X(j+1)
+// (which overwrites P_X(j)) runs after PV_X(j), and its completion also means PV_X(j) is done.
 //
 // The running max is only moved when a block's max exceeds it by more than 2^8 in the exp2
 // domain; the final O / l uses the same reference max for both, so the result is the same
@@ -43,26 +53,38 @@ template <int D>
 struct FwdLayout {
   static constexpr int TILE = 128 * D * 2;    // bytes of one 128-row bf16 tile (Q, K or V)
   static constexpr int SUB = 128 * 128;       // one 64-column (128-byte) swizzle panel of a tile
-  static constexpr int STAGES = (D == 128) ? 3 : 4;
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE;
-  static constexpr int V_OFF = K_OFF + STAGES * TILE;
-  static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
-  static constexpr int NBARS = 1 + 3 * STAGES + 2 + 2 + 2 + 1 + 1;
+  static constexpr int KST = (D == 128) ? 3 : 4;   // K ring depth (K is needed one MMA earlier than V)
+  static constexpr int VST = (D == 128) ? 2 : 4;   // V ring depth
+  static constexpr int QA_OFF = 0;
+  static constexpr int QB_OFF = QA_OFF + TILE;
+  static constexpr int K_OFF = QB_OFF + TILE;
+  static constexpr int V_OFF = K_OFF + KST * TILE;
+  static constexpr int BAR_OFF = V_OFF + VST * TILE;
+  // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2][2], o_fin[2], fin
+  static constexpr int NBARS = 1 + 2 * KST + 2 * VST + 2 + 4 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
-  static constexpr int S_COL0 = 0, S_COL1 = 128, O_COL = 256, P_COL0 = 256 + D, P_COL1 = 256 + D + 64;
+  __device__ static constexpr int s_col(int x) { return 128 * x; }         // S_A, S_B
+  __device__ static constexpr int o_col(int x) { return 256 + D * x; }     // O_A, O_B
   static constexpr int TMEM_COLS = 512;
-  static_assert(P_COL1 + 64 <= TMEM_COLS, "TMEM budget");
+  static_assert(256 + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
 
+// Exponentials of one pair of scores: p = 2^(s * sl2 - m).
+__device__ __forceinline__ uint64_t exp2_pair(uint32_t s0, uint32_t s1, uint64_t sl2x2, uint64_t negm2) {
+  const uint64_t x = f2_fma(f2_make(__uint_as_float(s0), __uint_as_float(s1)), sl2x2, negm2);
+  float x0, x1;
+  f2_split(x, x0, x1);
+  return f2_make(ex2_approx(x0), ex2_approx(x1));
+}
+
 template <int D, bool DROPOUT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using L = FwdLayout<D>;
-  constexpr int STAGES = L::STAGES;
+  constexpr int KST = L::KST, VST = L::VST;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if ((smem_u32(smem) & 1023u) != 0) {   // 128-byte swizzle atoms need 1024-byte alignment
@@ -72,45 +94,50 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + STAGES;
-  uint64_t* kv_empty = v_full + STAGES;
-  uint64_t* s_full = kv_empty + STAGES;
-  uint64_t* s_empty = s_full + 2;
-  uint64_t* p_full = s_empty + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* fin = o_done + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* s_full = v_empty + VST;   // [2]: tile A, tile B
+  uint64_t* p_full = s_full + 2;      // [2][2]: tile, half of the keys
+  uint64_t* o_fin = p_full + 4;
+  uint64_t* fin = o_fin + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
-  // ---- work item: longest causal rows first
-  const int qt = p.n_qtiles - 1 - int(blockIdx.x);
+  // ---- work item: query tiles 2i (A) and 2i+1 (B) of head bh; longest causal pairs first
+  const int pair = int(gridDim.x) - 1 - int(blockIdx.x);
   const int bh = blockIdx.y;
   const int b = bh / p.H;
-  const int q0 = qt * 128;
-  int kv_end = p.N;
-  if (p.key_lens != nullptr) kv_end = min(kv_end, max(p.key_lens[b], 0));
-  if (p.causal) kv_end = min(kv_end, q0 + 128);
-  const int n_kv = (kv_end + 127) / 128;
+  int kv_lim = p.N;
+  if (p.key_lens != nullptr) kv_lim = min(kv_lim, max(p.key_lens[b], 0));
+  // per tile x: first query row, key limit, number of 128-key blocks
+  auto tile_q0 = [&](int x) { return (2 * pair + x) * 128; };
+  auto tile_kv_end = [&](int x) { return p.causal ? min(kv_lim, tile_q0(x) + 128) : kv_lim; };
+  auto tile_n_kv = [&](int x) { return tile_q0(x) < p.N ? (tile_kv_end(x) + 127) / 128 : 0; };
+  const int n_max = max(tile_n_kv(0), tile_n_kv(1));
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VST; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);
-      mbar_init(&p_full[s], 4);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[2 * x], 4);
+      mbar_init(&p_full[2 * x + 1], 4);
+      mbar_init(&o_fin[x], 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -120,122 +147,158 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.wait_ns, abort_flag};
 
-  if (warp == 4) {
-    // =========================================================== producer
-    if (lane == 0 && n_kv > 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(q_full, L::TILE);
+  // Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
+  // 128 x (216 + 216 + 72) = 64512.  Each role lowers or raises its budget first thing.
+  if (warp == 11) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+  } else if (warp == 8 || warp == 10) {
+    // =========================================================== producers: warp 8 Q + K, warp 10 V
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+    const bool is_k = (warp == 8);
+    if (lane == 0 && n_max > 0) {
+      const int NS = is_k ? KST : VST;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      uint8_t* ring = smem + (is_k ? L::K_OFF : L::V_OFF);
+      prefetch_tmap(map);
+      if (is_k) {
+        prefetch_tmap(&tm_q);
+        mbar_arrive_expect_tx(q_full, 2 * L::TILE);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(smem + L::Q_OFF + c * L::SUB, &tm_q, q_full, c * 64, q0, bh);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(smem + L::QA_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(0), bh);
+          tma_load_3d(smem + L::QB_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(1), bh);
+        }
+      }
       int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % STAGES;
-        if (j >= STAGES && !mbar_wait(&kv_empty[st], ((j / STAGES) - 1) & 1, wc)) break;
+      for (int j = 0; j < n_max; ++j) {
+        const int st = j % NS;
+        if (j >= NS && !mbar_wait(&empty[st], ((j / NS) - 1) & 1, wc)) break;
         if ((p.debug_flags & 1) && j == 0) break;   // test hook: never deliver block 0
-        mbar_arrive_expect_tx(&k_full[st], L::TILE);
+        mbar_arrive_expect_tx(&full[st], L::TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::K_OFF + st * L::TILE + c * L::SUB, &tm_k, &k_full[st], c * 64, j * 128, bh);
-        mbar_arrive_expect_tx(&v_full[st], L::TILE);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::V_OFF + st * L::TILE + c * L::SUB, &tm_v, &v_full[st], c * 64, j * 128, bh);
+          tma_load_3d(ring + st * L::TILE + c * L::SUB, map, &full[st], c * 64, j * 128, bh);
         issued = j + 1;
       }
       // every copy this thread started must land before the CTA releases its shared memory
-      mbar_drain(q_full, 0, p.wait_ns);
-      for (int j = max(0, issued - STAGES); j < issued; ++j) {
-        mbar_drain(&k_full[j % STAGES], (j / STAGES) & 1, p.wait_ns);
-        mbar_drain(&v_full[j % STAGES], (j / STAGES) & 1, p.wait_ns);
-      }
+      if (is_k) mbar_drain(q_full, 0, p.wait_ns);
+      for (int j = max(0, issued - NS); j < issued; ++j) mbar_drain(&full[j % NS], (j / NS) & 1, p.wait_ns);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // =========================================================== MMA issuer
-    if (lane == 0 && n_kv > 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+    if (lane == 0 && n_max > 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
       constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
-      const uint32_t q_base = smem_u32(smem + L::Q_OFF);
-      auto issue_pv = [&](int t) -> bool {
-        const int st = t % STAGES, sb = t & 1;
-        if (!mbar_wait(&p_full[sb], (t >> 1) & 1, wc)) return false;
-        if (!mbar_wait(&v_full[st], (t / STAGES) & 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + L::V_OFF + st * L::TILE);
-        const uint32_t p_col = sb ? L::P_COL1 : L::P_COL0;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 swizzle atoms of V
-          mma_ts(tmem + L::O_COL, tmem + p_col + kk * 8, sdesc_sw128(v_base + kk * 2048, L::SUB, 1024), kIdPV,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&kv_empty[st]);
-        mma_commit(o_done);
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, wc);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j % STAGES, sb = j & 1;
-        if (!mbar_wait(&k_full[st], (j / STAGES) & 1, wc)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&s_empty[sb], ((j - 2) >> 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(smem + L::K_OFF + st * L::TILE);
-        const uint32_t s_col = sb ? L::S_COL1 : L::S_COL0;
+      const int n_a = tile_n_kv(0), n_b = tile_n_kv(1);
+      auto issue_s = [&](int x, int j) {   // S_x(j) = Q_x K_j^T
+        const uint32_t q_base = smem_u32(smem + (x ? L::QB_OFF : L::QA_OFF));
+        const uint32_t k_base = smem_u32(smem + L::K_OFF + (j % KST) * L::TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
           const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
-          mma_ss(tmem + s_col, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024), kIdS,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tmem + L::s_col(x), sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                 kIdS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        mma_commit(&s_full[x]);
+      };
+      auto issue_pv_half = [&](int x, int j, int h) {   // O_x += P_x(j)[keys of half h] V_j[same keys]
+        const uint32_t v_base = smem_u32(smem + L::V_OFF + (j % VST) * L::TILE);
+#pragma unroll
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
+          mma_ts(tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_sw128(v_base + kk * 2048, L::SUB, 1024),
+                 kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
+      if (ok) {
+        tc_fence_after();
+        if (n_a > 0) issue_s(0, 0);
+        if (n_b > 0) issue_s(1, 0);
+        mma_commit(&k_empty[0]);
       }
-      if (ok) issue_pv(n_kv - 1);
+      for (int j = 0; ok && j < n_max; ++j) {
+        if (!mbar_wait(&v_full[j % VST], (j / VST) & 1, wc)) { ok = false; break; }
+        const bool more = j + 1 < n_max;
+        bool have_k = false;   // K_{j+1} resident
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int n_x = x ? n_b : n_a;
+          if (j >= n_x) continue;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(&p_full[2 * x + h], j & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv_half(x, j, h);
+          }
+          if (!ok) break;
+          if (j + 1 < n_x) {
+            if (!have_k) {
+              if (!mbar_wait(&k_full[(j + 1) % KST], ((j + 1) / KST) & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+              have_k = true;
+            }
+            issue_s(x, j + 1);
+          } else {
+            mma_commit(&o_fin[x]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&v_empty[j % VST]);                  // V_j: both tiles' PV issued
+        if (more) mma_commit(&k_empty[(j + 1) % KST]);  // K_{j+1}: both tiles' S issued
+      }
       mma_commit(fin);   // completes when every MMA issued above has finished
       mbar_drain(fin, 0, p.wait_ns);
     }
     __syncwarp();
   } else {
-    // =========================================================== softmax / epilogue (warps 0-3)
-    const int r = tid;
-    const int q_row = q0 + r;
-    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    // =========================================================== softmax / epilogue (warps 0-7)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
+    const int x = warp >> 2;   // tile
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int q0x = tile_q0(x);
+    const int q_row = q0x + r;
+    const int n = tile_n_kv(x);
+    const int kv_x = tile_kv_end(x);
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t s_addr = lane_base + L::s_col(x);
+    const uint32_t o_addr = lane_base + L::o_col(x);
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_make(sl2, sl2);
     const uint64_t drop_row = (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * uint64_t(p.N);
     float m_ref = -INFINITY;   // reference max, exp2 domain
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (j >> 1) & 1, wc)) { ok = false; break; }
+    for (int j = 0; j < n; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, wc))) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
-      {
-        const uint32_t s_addr = lane_base + (sb ? L::S_COL1 : L::S_COL0);
-        tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        tmem_ld_wait();
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_ld_wait();
+#pragma unroll
+      for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
 
       const int k0 = j * 128;
-      if ((k0 + 128 > kv_end) || (p.causal && k0 + 128 > q0)) {   // block straddles a mask edge
-        const int lim = min(kv_end, p.causal ? q_row + 1 : kv_end) - k0;   // columns < lim are kept
+      const bool masked = (k0 + 128 > kv_x) || (p.causal && k0 + 128 > q0x);   // block straddles a mask edge
+      if (masked) {
+        const int lim = min(kv_x, p.causal ? q_row + 1 : kv_x) - k0;   // columns < lim are kept
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      for (int c = 0; c < 128; c += 8)
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          mxv[u] = max3f(mxv[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
+      const float mx = fmaxf(max3f(mxv[0], mxv[1], mxv[2]), mxv[3]);
       const float m_cand = mx * sl2;
       float alpha = 1.f;
       if (m_cand > m_ref + kRescaleThreshold) {
@@ -243,66 +306,65 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         m_ref = m_cand;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float rs = 0.f;
-      uint32_t pk[64];
+      const uint64_t negm2 = f2_make(-m_use, -m_use);
+      uint64_t rs2 = f2_make(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), sl2, -m_use));
-        float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -m_use));
-        rs += p0 + p1;
-        if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
-          const uint64_t ctr = drop_row + uint64_t(k0 + 2 * c);
-          p0 = dropout_keep(p.seed, ctr, p.drop_thr) ? p0 : 0.f;
-          p1 = dropout_keep(p.seed, ctr + 1, p.drop_thr) ? p1 : 0.f;
+      for (int h = 0; h < 2; ++h) {   // two halves of 64 keys; the MMA takes each half as soon as it is ready
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = 32 * h + e;   // pair index: keys 2c, 2c+1
+          const uint64_t pp = exp2_pair(sr[2 * c], sr[2 * c + 1], sl2x2, negm2);
+          rs2 = f2_add(rs2, pp);
+          float p0, p1;
+          f2_split(pp, p0, p1);
+          if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
+            const uint64_t ctr = drop_row + uint64_t(k0 + 2 * c);
+            p0 = dropout_keep(p.seed, ctr, p.drop_thr) ? p0 : 0.f;
+            p1 = dropout_keep(p.seed, ctr + 1, p.drop_thr) ? p1 : 0.f;
+          }
+          pk[e] = pack_bf16x2(p0, p1);
         }
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      // PV of the previous block must be complete: it frees this P buffer (used two blocks ago)
-      // and makes O final up to block j-1 before it is rescaled.
-      if (j >= 1) {
-        if (!mbar_wait(o_done, (j - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-      }
-      {
-        const uint32_t p_addr = lane_base + (sb ? L::P_COL1 : L::P_COL0);
-        tmem_st32(p_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(p_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      }
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // P over the score columns already read; O already holds PV up to block j-1
+        tmem_st32(s_addr + 32 * h, pk);
+        if (h == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(lane_base + L::O_COL + c * 32, orr);
-          tmem_ld_wait();
-          reg_fence32(orr);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(o_addr + c * 32, orr);
+            tmem_ld_wait();
+            reg_fence32(orr);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-          tmem_st32(lane_base + L::O_COL + c * 32, orr);
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st32(o_addr + c * 32, orr);
+          }
         }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[2 * x + h]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-      l = l * alpha + rs;
+      float rs0, rs1;
+      f2_split(rs2, rs0, rs1);
+      l = l * alpha + (rs0 + rs1);
     }
 
     // ---- epilogue: O / l -> bf16, lse = (m + log2 l) * ln 2
     const bool row_valid = q_row < p.N;
     __nv_bfloat16* orow = p.o + (uint64_t(bh) * uint64_t(p.N) + uint64_t(row_valid ? q_row : 0)) * D;
-    if (n_kv == 0) {
+    if (n == 0) {
       if (row_valid) {
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
         p.lse[uint64_t(bh) * p.N + q_row] = -INFINITY;
       }
-    } else if (ok && mbar_wait(o_done, (n_kv - 1) & 1, wc)) {
+    } else if (ok && __all_sync(0xffffffffu, mbar_wait(&o_fin[x], 0, wc))) {
       tc_fence_after();
       const float inv_l = l > 0.f ? (DROPOUT ? p.drop_scale : 1.f) / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
-        tmem_ld32(lane_base + L::O_COL + c * 32, orr);
+        tmem_ld32(o_addr + c * 32, orr);
         tmem_ld_wait();
         reg_fence32(orr);
         uint32_t packed[16];
@@ -323,7 +385,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   // ---- teardown: every role has drained its asynchronous work
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
