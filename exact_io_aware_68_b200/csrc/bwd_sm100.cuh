@@ -16,18 +16,22 @@
 //
 // Main kernel roles (12 warps, three warpgroups with their own register budgets):
 //   warps 0-3  compute (248 registers): thread r owns key row r (TMEM lane r).
-//              P^T = exp2(S^T tau log2e - lse2) (packed f32x2 arithmetic), masks, dropout; (P*Z)^T as bf16 into TMEM (dV
-//              takes 1/(1-p) at the end); dS^T = P^T (dP^T Z/(1-p) - D) as bf16 into TMEM (for dK)
-//              and into shared memory (one tile read by the dQ MMA as an MN-major operand); dV epilogue
+//              P^T = exp2(S^T tau log2e - lse2) (packed f32x2 arithmetic), masks, dropout; (P*Z)^T as
+//              bf16 into TMEM over the first 64 score columns (dV takes 1/(1-p) at the end);
+//              dS^T = P^T (dP^T Z/(1-p) - D) as bf16 into shared memory: one swizzled tile that the
+//              dK MMA reads as a K-major A operand and the dQ MMA as an MN-major B operand; dV epilogue
 //   warps 4-7  dQ (168 registers): read the dQ^T tile from TMEM (lane = feature, column = query),
-//              stage it in shared memory (the dS buffer, free once the dQ MMA is done) and add it to
-//              the fp32 accumulator with TMA bulk reductions, one per warp; dK epilogue
-//   warp 8     producer: TMA K, V once; Q, dO per query tile (STAGES deep); lse and D per tile
-//   warp 9     MMA issuer; warps 10-11 idle (88 registers for warps 8-11)
-// TMEM (512 columns): ST [0,128) S^T then (P*Z)^T in [0,64); DPT [128,256) dP^T then dS^T in
-// [128,192); dV [256,256+D); dK [256+D,256+2D).  dQ^T = K^T dS^T: D=64 -> M=64, N=128 in
-// [384,512); D=128 -> two N=64 halves in [64,128) and [192,256), so the next S^T / dP^T waits
-// until dQ^T has been read.
+//              stage it in its own shared-memory buffer and add it to the fp32 accumulator with TMA
+//              bulk reductions, one per warp, running in the background; dK epilogue
+//   warp 8     producer: TMA K, V once; Q (2 deep) and dO (1 deep at D=128, 2 at D=64) per query
+//              tile
+//   warp 9     MMA issuer; warp 10 loads lse and D per query tile; warp 11 idle
+//              (88 registers for warps 8-11)
+// TMEM (512 columns): ST [0,128) S^T, then (P*Z)^T in [0,64); DPT [128,256) dP^T, then dQ^T;
+// dV [256,256+D); dK [256+D,256+2D).  MMA order per query tile t:
+//   dV_t, S_{t+1}, dQ_t, dK_t, dP_{t+1}
+// so S_{t+1} is ready when the compute warps finish dS_t, and only dV_t (needs P_t) and dQ_t
+// (needs dS_t) wait on them.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -110,27 +114,29 @@ template <int D>
 struct BwdLayout {
   static constexpr int TILE = 128 * D * 2;
   static constexpr int SUB = 128 * 128;
-  static constexpr int STAGES = (D == 128) ? 2 : 3;
+  static constexpr int QS = 2;                       // Q ring (and per-tile statistics) depth
+  static constexpr int DS = (D == 128) ? 1 : 2;      // dO ring depth: dO_{t+1} is needed only after dV_t
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
   static constexpr int Q_OFF = V_OFF + TILE;
-  static constexpr int DO_OFF = Q_OFF + STAGES * TILE;
-  static constexpr int DS_OFF = DO_OFF + STAGES * TILE;      // 128 keys x 128 queries bf16, 2 panels
-  static constexpr int STAT_OFF = DS_OFF + 2 * SUB;           // per stage: lse2[128], D[128]
-  static constexpr int BAR_OFF = STAT_OFF + STAGES * 1024;
-  // kv_full, q_full[S], do_full[S], stat_full[S], q_empty[S], s_full, dp_full, p_full, ds_full,
-  // dq_full, dq_empty, ds_free, fin
-  static constexpr int NBARS = 1 + 4 * STAGES + 8;
+  static constexpr int DO_OFF = Q_OFF + QS * TILE;
+  static constexpr int DS_OFF = DO_OFF + DS * TILE;          // 128 keys x 128 queries bf16, 2 panels
+  static constexpr int STG_OFF = DS_OFF + 2 * SUB;            // dQ staging for the bulk reductions
+  static constexpr int STAT_OFF = STG_OFF + 32768;            // per stage: -lse2[128], -D[128]
+  static constexpr int BAR_OFF = STAT_OFF + QS * 1024;
+  // kv_full, q_full[QS], q_empty[QS], stat_full[QS], do_full[DS], do_empty[DS], s_full, dp_full,
+  // p_full, ds_full, dq_full, dq_empty, dk_done, fin
+  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ST_COL = 0, DPT_COL = 128, DV_COL = 256, DK_COL = 256 + D;
   static constexpr int TMEM_COLS = 512;
-  // dQ staging (in the dS buffer): per warp and round, QPR queries x FPW features of fp32
+  // dQ staging: per warp and round, QPR queries x FPW features of fp32 (8 KB)
   static constexpr int FPW = (D == 128) ? 32 : 16;     // features per warp (TMEM lanes with data)
   static constexpr int QPR = (D == 128) ? 64 : 128;    // queries per reduction round
   static constexpr int ROUNDS = 128 / QPR;
-  static constexpr int STAGE_BYTES = QPR * FPW * 4;    // 8 KB per warp
-  static_assert(4 * STAGE_BYTES <= 2 * SUB, "dQ staging fits in the dS buffer");
+  static constexpr int STAGE_BYTES = QPR * FPW * 4;
+  static_assert(4 * STAGE_BYTES <= 32768, "dQ staging fits its buffer");
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
@@ -154,7 +160,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdLayout<D>;
-  constexpr int STAGES = L::STAGES;
+  constexpr int QS = L::QS, DS = L::DS;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -164,17 +170,18 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
-  uint64_t* do_full = q_full + STAGES;
-  uint64_t* stat_full = do_full + STAGES;
-  uint64_t* q_empty = stat_full + STAGES;
-  uint64_t* s_full = q_empty + STAGES;
+  uint64_t* q_empty = q_full + QS;
+  uint64_t* stat_full = q_empty + QS;
+  uint64_t* do_full = stat_full + QS;
+  uint64_t* do_empty = do_full + DS;
+  uint64_t* s_full = do_empty + DS;
   uint64_t* dp_full = s_full + 1;
   uint64_t* p_full = dp_full + 1;
   uint64_t* ds_full = p_full + 1;
   uint64_t* dq_full = ds_full + 1;
   uint64_t* dq_empty = dq_full + 1;
-  uint64_t* ds_free = dq_empty + 1;
-  uint64_t* fin = ds_free + 1;
+  uint64_t* dk_done = dq_empty + 1;
+  uint64_t* fin = dk_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
@@ -191,11 +198,14 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&do_full[s], 1);
-      mbar_init(&stat_full[s], 32);
       mbar_init(&q_empty[s], 1);
+      mbar_init(&stat_full[s], 32);
+    }
+    for (int s = 0; s < DS; ++s) {
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -203,7 +213,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(ds_full, 4);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 4);
-    mbar_init(ds_free, 4);
+    mbar_init(dk_done, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -222,12 +232,35 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   // Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
   // 128 x (248 + 168 + 88) = 64512.  Each role lowers or raises its budget first thing.
-  if (warp >= 10) {
+  if (warp == 11) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+  } else if (warp == 10) {
+    // =========================================================== per-tile statistics
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    for (int t = 0; t < n_iter; ++t) {
+      const int sq = t % QS;
+      const int qrow0 = (q_first + t) * 128;
+      // the stage is reused once dK of tile t-QS (after every read of its statistics) is done
+      if (t >= QS && !warp_wait(&q_empty[sq], ((t / QS) - 1) & 1, wc)) break;
+      // negated: -lse in the exp2 domain and -D
+      float* st_l = stat + sq * 256;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = lane * 4 + e;
+        const int q = qrow0 + c;
+        float lv = 0.f, dv = 0.f;
+        if (q < p.N) {
+          lv = -p.lse[row_base + q] * kLog2e;
+          dv = -p.dvec[row_base + q];
+        }
+        st_l[c] = lv;
+        st_l[128 + c] = dv;
+      }
+      mbar_arrive(&stat_full[sq]);
+    }
   } else if (warp == 8) {
     // =========================================================== producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
-    int issued = 0;
     if (n_iter > 0) {
       if (lane == 0) {
         prefetch_tmap(&tm_q);
@@ -242,43 +275,32 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tma_load_3d(smem + L::V_OFF + c * L::SUB, &tm_v, kv_full, c * 64, k0, bh);
         }
       }
+      int issued_q = 0, issued_do = 0;
       for (int t = 0; t < n_iter; ++t) {
-        const int st = t % STAGES;
+        const int sq = t % QS, sd = t % DS;
         const int qrow0 = (q_first + t) * 128;
-        if (t >= STAGES && !warp_wait(&q_empty[st], ((t / STAGES) - 1) & 1, wc)) break;
+        if (t >= QS && !warp_wait(&q_empty[sq], ((t / QS) - 1) & 1, wc)) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full[st], L::TILE);
+          mbar_arrive_expect_tx(&q_full[sq], L::TILE);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + L::Q_OFF + st * L::TILE + c * L::SUB, &tm_q, &q_full[st], c * 64, qrow0, bh);
-          mbar_arrive_expect_tx(&do_full[st], L::TILE);
+            tma_load_3d(smem + L::Q_OFF + sq * L::TILE + c * L::SUB, &tm_q, &q_full[sq], c * 64, qrow0, bh);
+        }
+        issued_q = t + 1;
+        if (t >= DS && !warp_wait(&do_empty[sd], ((t / DS) - 1) & 1, wc)) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&do_full[sd], L::TILE);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + L::DO_OFF + st * L::TILE + c * L::SUB, &tm_do, &do_full[st], c * 64, qrow0, bh);
+            tma_load_3d(smem + L::DO_OFF + sd * L::TILE + c * L::SUB, &tm_do, &do_full[sd], c * 64, qrow0, bh);
         }
-        // per-query statistics of this tile, negated: -lse in the exp2 domain and -D
-        float* st_l = stat + st * 256;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = lane * 4 + e;
-          const int q = qrow0 + c;
-          float lv = 0.f, dv = 0.f;
-          if (q < p.N) {
-            lv = -p.lse[row_base + q] * kLog2e;
-            dv = -p.dvec[row_base + q];
-          }
-          st_l[c] = lv;
-          st_l[128 + c] = dv;
-        }
-        mbar_arrive(&stat_full[st]);
-        issued = t + 1;
+        issued_do = t + 1;
       }
       if (lane == 0) {
         mbar_drain(kv_full, 0, p.wait_ns);
-        for (int t = max(0, issued - STAGES); t < issued; ++t) {
-          mbar_drain(&q_full[t % STAGES], (t / STAGES) & 1, p.wait_ns);
-          mbar_drain(&do_full[t % STAGES], (t / STAGES) & 1, p.wait_ns);
-        }
+        for (int t = max(0, issued_q - QS); t < issued_q; ++t) mbar_drain(&q_full[t % QS], (t / QS) & 1, p.wait_ns);
+        for (int t = max(0, issued_do - DS); t < issued_do; ++t)
+          mbar_drain(&do_full[t % DS], (t / DS) & 1, p.wait_ns);
       }
     }
     __syncwarp();
@@ -286,22 +308,16 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // =========================================================== MMA issuer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
     if (lane == 0 && n_iter > 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);             // K (V) and Q (dO) K-major
-      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);                // A in TMEM, B MN-major
-      constexpr uint32_t kIdQ = idesc_bf16(D, D == 128 ? 64 : 128, true, true);  // K^T, dS^T: both MN-major
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (V) and Q (dO) K-major
+      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A K-major, B MN-major
+      constexpr uint32_t kIdQ = idesc_bf16(D, 128, true, true);       // dQ^T: K^T, dS^T both MN-major
       const uint32_t k_base = smem_u32(smem + L::K_OFF);
       const uint32_t v_base = smem_u32(smem + L::V_OFF);
       const uint32_t ds_base = smem_u32(smem + L::DS_OFF);
-      bool ok = mbar_wait(kv_full, 0, wc);
-      for (int t = 0; ok && t < n_iter; ++t) {
-        const int st = t % STAGES;
-        const uint32_t sp = (t / STAGES) & 1;
-        const uint32_t q_base = smem_u32(smem + L::Q_OFF + st * L::TILE);
-        const uint32_t do_base = smem_u32(smem + L::DO_OFF + st * L::TILE);
-        if (!mbar_wait(&q_full[st], sp, wc)) { ok = false; break; }
-        if (D == 128 && t >= 1 && !mbar_wait(dq_empty, (t - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        // S^T = K Q^T  (M = 128 keys, N = 128 queries, K = D)
+      auto q_at = [&](int t) { return smem_u32(smem + L::Q_OFF + (t % QS) * L::TILE); };
+      auto do_at = [&](int t) { return smem_u32(smem + L::DO_OFF + (t % DS) * L::TILE); };
+      auto issue_s = [&](int t) {   // S^T = K Q_t^T  (M = 128 keys, N = 128 queries, K = D)
+        const uint32_t q_base = q_at(t);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
@@ -309,9 +325,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                  kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full);
-        // dP^T = V dO^T
-        if (!mbar_wait(&do_full[st], sp, wc)) { ok = false; break; }
-        tc_fence_after();
+      };
+      auto issue_dp = [&](int t) {   // dP^T = V dO_t^T
+        const uint32_t do_base = do_at(t);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
@@ -319,39 +335,55 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                  kIdS, kk > 0 ? 1u : 0u);
         }
         mma_commit(dp_full);
-        // dV += (P*Z)^T dO   (A = (P*Z)^T in TMEM, B = dO MN-major: N = D, K = queries)
+      };
+      bool ok = mbar_wait(kv_full, 0, wc) && mbar_wait(&q_full[0], 0, wc);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        ok = mbar_wait(&do_full[0], 0, wc);
+        if (ok) {
+          tc_fence_after();
+          issue_dp(0);
+        }
+      }
+      for (int t = 0; ok && t < n_iter; ++t) {
+        const bool more = t + 1 < n_iter;
+        // dV += (P*Z)^T dO_t   (A = (P*Z)^T in TMEM, B = dO MN-major: N = D, K = queries)
         if (!mbar_wait(p_full, t & 1, wc)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_sw128(do_base + kk * 2048, L::SUB, 1024), kIdG,
+          mma_ts(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_sw128(do_at(t) + kk * 2048, L::SUB, 1024), kIdG,
                  (t > 0 || kk > 0) ? 1u : 0u);
-        // dQ^T tile = K^T dS^T   (M = D features, K = 128 keys, N = queries), issued before dK so
-        // that the dQ warps read it out while dK runs
-        if (!mbar_wait(ds_full, t & 1, wc)) { ok = false; break; }
-        if (D == 64 && t >= 1 && !mbar_wait(dq_empty, (t - 1) & 1, wc)) { ok = false; break; }
-        tc_fence_after();
-        if (D == 128) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + (h == 0 ? 64u : 192u), sdesc_sw128(k_base + kk * 2048, L::SUB, 1024),
-                     sdesc_sw128(ds_base + h * L::SUB + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
-          }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + 384u, sdesc_sw128(k_base + kk * 2048, L::SUB, 1024),
-                   sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        mma_commit(&do_empty[t % DS]);   // dO_t: last read by dV_t
+        // S_{t+1} over the (P*Z)^T that dV_t has just been given (MMAs run in issue order)
+        if (more) {
+          if (!mbar_wait(&q_full[(t + 1) % QS], ((t + 1) / QS) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(t + 1);
         }
-        mma_commit(dq_full);
-        // dK += dS^T Q
+        // dQ^T = K^T dS^T into the dP^T columns (already read)   (M = D, N = 128 queries, K = 128 keys)
+        if (!mbar_wait(ds_full, t & 1, wc)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::DK_COL, tmem + L::DPT_COL + kk * 8, sdesc_sw128(q_base + kk * 2048, L::SUB, 1024), kIdG,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&q_empty[st]);
+          mma_ss(tmem + L::DPT_COL, sdesc_sw128(k_base + kk * 2048, L::SUB, 1024),
+                 sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        mma_commit(dq_full);
+        // dK += dS^T Q_t   (A = dS^T from shared memory, K-major: rows = keys, 16 queries per step)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::DK_COL, sdesc_sw128(ds_base + (kk >> 2) * L::SUB + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(q_at(t) + kk * 2048, L::SUB, 1024), kIdG, (t > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(dk_done);             // the dS tile is free again
+        mma_commit(&q_empty[t % QS]);    // Q_t: last read by dK_t
+        // dP_{t+1} once the dQ warps have read dQ^T out of those columns
+        if (more) {
+          if (!mbar_wait(dq_empty, t & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&do_full[(t + 1) % DS], ((t + 1) / DS) & 1, wc)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(t + 1);
+        }
       }
       mma_commit(fin);
       mbar_drain(fin, 0, p.wait_ns);
@@ -367,12 +399,12 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     bool ok = true;
     uint8_t* ds_smem = smem + L::DS_OFF;
     for (int t = 0; t < n_iter; ++t) {
-      const int st = t % STAGES;
+      const int sq = t % QS;
       const int qrow0 = (q_first + t) * 128;
-      const float* st_l = stat + st * 256;
+      const float* st_l = stat + sq * 256;
       const bool need_mask = (k0 + 128 > kv_end) || (qrow0 + 128 > p.N) || (p.causal && q_first + t == kt);
       if (!warp_wait(s_full, t & 1, wc)) { ok = false; break; }
-      if (!warp_wait(&stat_full[st], (t / STAGES) & 1, wc)) { ok = false; break; }
+      if (!warp_wait(&stat_full[sq], (t / QS) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       // ---- P^T = exp2(S^T tau log2e - lse2): one pass over the 128 query columns
       float pr[128];
@@ -436,8 +468,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
       // ---- dS^T = P^T * (dP^T Z/(1-p) - D), two halves of 64 query columns
       if (!warp_wait(dp_full, t & 1, wc)) { ok = false; break; }
-      // the dQ warps have finished with the shared dS buffer (the last dQ MMA and its reductions)
-      if (t >= 1 && !warp_wait(ds_free, (t - 1) & 1, wc)) { ok = false; break; }
+      // the dS tile is free: dQ_{t-1} and dK_{t-1} have read it
+      if (t >= 1 && !warp_wait(dk_done, (t - 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
@@ -462,7 +494,6 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           f2_split(f2_mul(f2_make(pr[c], pr[c + 1]), f2_add(f2_make(dpa, dpb), nd2[c >> 1])), da, db);
           pk[e] = pack_bf16x2(da, db);
         }
-        tmem_st32(lane_base + L::DPT_COL + 32 * hh, pk);
         // dS (queries contiguous) into the 128-byte-swizzled panel hh: row = key r, 16-byte chunks
 #pragma unroll
         for (int chunk = 0; chunk < 8; ++chunk) {   // 8 queries per 16-byte chunk
@@ -471,8 +502,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       }
       fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
-      tmem_st_wait();
-      tc_fence_before();
+      tc_fence_before();          // (the dP^T loads above precede the dQ MMA that overwrites them)
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
     }
@@ -505,14 +535,15 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
   } else {
     // =========================================================== dQ + dK epilogue (warps 4-7)
-    // TMEM holds dQ^T: lane = feature, column = query.  D=128: feature 32*quarter + lane;
-    // D=64 (M=64 layout): feature 16*quarter + lane on lanes 0-15.  Each warp stages its
-    // features for QPR queries in its 8 KB slice of the dS buffer ([query][feature], fp32) and
-    // adds that box to the accumulator with one TMA bulk reduction.
+    // TMEM holds dQ^T in the dP^T columns: lane = feature, column = query.  D=128: feature
+    // 32*quarter + lane; D=64 (M=64 layout): feature 16*quarter + lane on lanes 0-15.  Each warp
+    // stages its features for QPR queries in its 8 KB slice of the staging buffer ([query][feature],
+    // fp32) and adds that box to the accumulator with one TMA bulk reduction; the reductions run
+    // in the background while the next tiles are computed.
     const int quarter = warp - 4;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
-    float* stage = reinterpret_cast<float*>(smem + L::DS_OFF + quarter * L::STAGE_BYTES);
+    float* stage = reinterpret_cast<float*>(smem + L::STG_OFF + quarter * L::STAGE_BYTES);
     const bool lane_ok = lane < L::FPW;
     bool ok = true;
     for (int t = 0; t < n_iter; ++t) {
@@ -520,28 +551,20 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (!warp_wait(dq_full, t & 1, wc)) { ok = false; break; }
       tc_fence_after();
       uint32_t g[128];
-      if (D == 128) {
-        tmem_ld32(lane_base + 64, *reinterpret_cast<uint32_t(*)[32]>(&g[0]));
-        tmem_ld32(lane_base + 96, *reinterpret_cast<uint32_t(*)[32]>(&g[32]));
-        tmem_ld32(lane_base + 192, *reinterpret_cast<uint32_t(*)[32]>(&g[64]));
-        tmem_ld32(lane_base + 224, *reinterpret_cast<uint32_t(*)[32]>(&g[96]));
-      } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + 384 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&g[32 * c]));
-      }
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(lane_base + L::DPT_COL + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&g[32 * c]));
       tmem_ld_wait();
 #pragma unroll
       for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&g[h * 32]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_empty);
-      // the dQ MMA has completed, so the dS buffer is free for staging
 #pragma unroll
       for (int rd = 0; rd < L::ROUNDS; ++rd) {
-        if (rd > 0) {   // the previous round's reduction must have read the staging slice
-          if (lane == 0) bulk_wait_read0();
-          __syncwarp();
-        }
+        // the previous reduction from this staging slice must have read it
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
         if (lane_ok) {
 #pragma unroll
           for (int c = 0; c < L::QPR; ++c) stage[c * L::FPW + lane] = __uint_as_float(g[rd * L::QPR + c]);
@@ -553,9 +576,6 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           bulk_commit();
         }
       }
-      if (lane == 0) bulk_wait_read0();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_free);
     }
     if (lane == 0) bulk_wait0();   // every reduction has completed before the kernel ends
     __syncwarp();
