@@ -136,6 +136,24 @@ fa_status check_workspace(void* ws, size_t bytes, int B, int H, int N, int d, Wo
   return FA_OK;
 }
 
+// Number of SMs of the current device (queried once per device).
+fa_status sm_count(int* out) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev >= 0 && dev < 64 && cache[dev].load() > 0) {
+    *out = cache[dev].load();
+    return FA_OK;
+  }
+  int n = 0;
+  e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess || n <= 0) return fail(FA_ERR_CUDA, "cudaDeviceGetAttribute(SM count): %s", cudaGetErrorString(e));
+  if (dev >= 0 && dev < 64) cache[dev].store(n);
+  *out = n;
+  return FA_OK;
+}
+
 template <typename K>
 fa_status set_smem(K kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -149,7 +167,11 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   using L = fa::FwdLayout<D>;
   fa_status st = set_smem(fa::fa_fwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
-  const dim3 grid((p.n_qtiles + 1) / 2, p.B * p.H);   // one CTA per pair of 128-row query tiles
+  // persistent: one CTA per SM (or fewer when there are fewer work items)
+  const long long items = (long long)p.n_pairs * p.B * p.H;
+  int sms = 0;
+  if ((st = sm_count(&sms)) != FA_OK) return st;
+  const dim3 grid(unsigned(items < sms ? items : sms));
   fa::fa_fwd_sm100_kernel<D, DROPOUT><<<grid, 384, L::BYTES, s>>>(mq, mk, mv, p);
   return launch_status("fa_fwd kernel launch");
 }
@@ -217,6 +239,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.H = H;
   p.N = N;
   p.n_qtiles = (N + 127) / 128;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.dropout = dropout_p > 0.f ? 1 : 0;

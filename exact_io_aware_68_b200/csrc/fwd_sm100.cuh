@@ -3,16 +3,19 @@
 // "Tiling и online softmax": m <- max(m, m_block), l and O re-expressed against the new m), so
 // the N x N score matrix never reaches HBM.
 //
-// One CTA computes two adjacent 128-row query tiles A and B of one (b, h) and loops over 128-key
-// blocks; both tiles share every K/V block.  Warp roles (three warpgroups):
+// Work item: two adjacent 128-row query tiles A and B of one (b, h); the item loops over 128-key
+// blocks and both tiles share every K/V block.  The grid is persistent (one CTA per SM): each CTA
+// takes the items of a heavy-first list in snake order (round r: CTA c takes item r*G + c, or
+// r*G + G-1-c on odd rounds), and its pipelines run on from one item into the next: the K/V rings
+// continue, the next Q tiles load as soon as the last S of an item has been issued, and the next
+// item's first S overlaps the epilogue of the previous one.  Warp roles (three warpgroups):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns query row r of its
 //              tile (= TMEM lane r); masks, exponentiates, writes P (bf16) over the tile's score
 //              columns, rescales O when needed, writes O and lse at the end
-//   warp 8     producer of both Q tiles and the K ring; warp 10 producer of the V ring
+//   warp 8     producer of the K ring, warp 10 of the V ring, warp 11 of the two Q tiles
 //   warp 9     MMA issuer, in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while one tile's
 //              softmax runs, the tensor core works on the other tile.  P is handed over in two
 //              halves of 64 keys, so the first half of PV runs while the second half of P is made.
-//   warp 11    idle
 // Softmax arithmetic: the scale-and-shift and the row sum use packed f32x2 operations and the row
 // max a tree of three-input maxima; every exponential goes to the MUFU unit (moving a share to a
 // polynomial on the FMA pipe was measured slower: the softmax is bound by instruction issue).
@@ -36,6 +39,7 @@ struct FwdParams {
   const int32_t* key_lens;     // [B] or null
   int B, H, N;
   int n_qtiles;
+  int n_pairs;                 // ceil(n_qtiles / 2): work items per head
   int causal;
   float scale_log2;            // tau * log2(e)
   int dropout;                 // 0 / 1
@@ -60,8 +64,9 @@ struct FwdLayout {
   static constexpr int K_OFF = QB_OFF + TILE;
   static constexpr int V_OFF = K_OFF + KST * TILE;
   static constexpr int BAR_OFF = V_OFF + VST * TILE;
-  // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2][2], o_fin[2], fin
-  static constexpr int NBARS = 1 + 2 * KST + 2 * VST + 2 + 4 + 2 + 1;
+  // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2][2],
+  // o_fin[2], o_free[2], fin
+  static constexpr int NBARS = 2 + 2 * KST + 2 * VST + 2 + 4 + 2 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   __device__ static constexpr int s_col(int x) { return 128 * x; }         // S_A, S_B
@@ -79,6 +84,17 @@ __device__ __forceinline__ uint64_t exp2_pair(uint32_t s0, uint32_t s1, uint64_t
   return f2_make(ex2_approx(x0), ex2_approx(x1));
 }
 
+__device__ __forceinline__ void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory"); }
+__device__ __forceinline__ void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory"); }
+
+// Item k of the heavy-first list: pair (longest causal pairs first) and head.
+__device__ __forceinline__ void fwd_item(int k, int n_pairs, int BH, int& pair, int& bh) {
+  pair = n_pairs - 1 - k / BH;
+  bh = k % BH;
+}
+// Item taken by CTA c of G in round r (snake order).
+__device__ __forceinline__ int fwd_snake(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
+
 template <int D, bool DROPOUT>
 __global__ void __launch_bounds__(384, 1)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -93,31 +109,40 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* k_full = q_empty + 1;
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + VST;
   uint64_t* s_full = v_empty + VST;   // [2]: tile A, tile B
   uint64_t* p_full = s_full + 2;      // [2][2]: tile, half of the keys
-  uint64_t* o_fin = p_full + 4;
-  uint64_t* fin = o_fin + 2;
+  uint64_t* o_fin = p_full + 4;       // [2]: all PV of the item done
+  uint64_t* o_free = o_fin + 2;       // [2]: the epilogue has read O
+  uint64_t* fin = o_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
-  // ---- work item: query tiles 2i (A) and 2i+1 (B) of head bh; longest causal pairs first
-  const int pair = int(gridDim.x) - 1 - int(blockIdx.x);
-  const int bh = blockIdx.y;
-  const int b = bh / p.H;
-  int kv_lim = p.N;
-  if (p.key_lens != nullptr) kv_lim = min(kv_lim, max(p.key_lens[b], 0));
-  // per tile x: first query row, key limit, number of 128-key blocks
-  auto tile_q0 = [&](int x) { return (2 * pair + x) * 128; };
-  auto tile_kv_end = [&](int x) { return p.causal ? min(kv_lim, tile_q0(x) + 128) : kv_lim; };
-  auto tile_n_kv = [&](int x) { return tile_q0(x) < p.N ? (tile_kv_end(x) + 127) / 128 : 0; };
-  const int n_max = max(tile_n_kv(0), tile_n_kv(1));
+  const int G = int(gridDim.x), cta = int(blockIdx.x);
+  const int BH = p.B * p.H;
+  const int n_items = p.n_pairs * BH;
+  // per item and tile x: first query row, key limit, number of 128-key blocks
+  auto kv_lim_of = [&](int bh) {
+    int lim = p.N;
+    if (p.key_lens != nullptr) lim = min(lim, max(p.key_lens[bh / p.H], 0));
+    return lim;
+  };
+  auto tile_q0 = [&](int pair, int x) { return (2 * pair + x) * 128; };
+  auto tile_kv_end = [&](int pair, int bh, int x) {
+    const int lim = kv_lim_of(bh);
+    return p.causal ? min(lim, tile_q0(pair, x) + 128) : lim;
+  };
+  auto tile_n_kv = [&](int pair, int bh, int x) {
+    return tile_q0(pair, x) < p.N ? (tile_kv_end(pair, bh, x) + 127) / 128 : 0;
+  };
 
   if (tid == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < KST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -131,6 +156,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(&p_full[2 * x], 4);
       mbar_init(&p_full[2 * x + 1], 4);
       mbar_init(&o_fin[x], 1);
+      mbar_init(&o_free[x], 4);
     }
     mbar_init(fin, 1);
     *abort_flag = 0;
@@ -148,106 +174,147 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const WaitCtl wc{p.wait_ns, abort_flag};
 
   // Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
-  // 128 x (216 + 216 + 72) = 64512.  Each role lowers or raises its budget first thing.
+  // 128 x (200 + 200 + 104) = 64512.  Each role lowers or raises its budget first thing.
   if (warp == 11) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+    // =========================================================== producer of the Q tiles
+    reg_dealloc();
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      int n_q = 0;          // Q pairs delivered
+      for (int r = 0;; ++r) {
+        const int k = fwd_snake(r, cta, G);
+        if (k >= n_items) break;
+        int pair, bh;
+        fwd_item(k, p.n_pairs, BH, pair, bh);
+        if (max(tile_n_kv(pair, bh, 0), tile_n_kv(pair, bh, 1)) == 0) continue;
+        // both Q tiles, once the previous item's last S has read the buffers
+        if (n_q >= 1 && !mbar_wait(q_empty, (n_q - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(q_full, 2 * L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(smem + L::QA_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(pair, 0), bh);
+          tma_load_3d(smem + L::QB_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(pair, 1), bh);
+        }
+        ++n_q;
+      }
+      if (n_q >= 1) mbar_drain(q_full, (n_q - 1) & 1, p.wait_ns);   // the last copies land before exit
+    }
+    __syncwarp();
   } else if (warp == 8 || warp == 10) {
-    // =========================================================== producers: warp 8 Q + K, warp 10 V
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+    // =========================================================== producers of the K (warp 8) and V (warp 10) rings
+    reg_dealloc();
     const bool is_k = (warp == 8);
-    if (lane == 0 && n_max > 0) {
+    if (lane == 0) {
       const int NS = is_k ? KST : VST;
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       const CUtensorMap* map = is_k ? &tm_k : &tm_v;
       uint8_t* ring = smem + (is_k ? L::K_OFF : L::V_OFF);
       prefetch_tmap(map);
-      if (is_k) {
-        prefetch_tmap(&tm_q);
-        mbar_arrive_expect_tx(q_full, 2 * L::TILE);
+      int g = 0;            // blocks delivered on this ring so far (all items)
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int k = fwd_snake(r, cta, G);
+        if (k >= n_items) break;
+        int pair, bh;
+        fwd_item(k, p.n_pairs, BH, pair, bh);
+        const int n_max = max(tile_n_kv(pair, bh, 0), tile_n_kv(pair, bh, 1));
+        for (int j = 0; j < n_max; ++j, ++g) {
+          const int st = g % NS;
+          if (g >= NS && !mbar_wait(&empty[st], ((g / NS) - 1) & 1, wc)) { ok = false; break; }
+          if ((p.debug_flags & 1) && g == 0) { ok = false; break; }   // test hook: never deliver block 0
+          mbar_arrive_expect_tx(&full[st], L::TILE);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + L::QA_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(0), bh);
-          tma_load_3d(smem + L::QB_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(1), bh);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(ring + st * L::TILE + c * L::SUB, map, &full[st], c * 64, j * 128, bh);
         }
       }
-      int issued = 0;
-      for (int j = 0; j < n_max; ++j) {
-        const int st = j % NS;
-        if (j >= NS && !mbar_wait(&empty[st], ((j / NS) - 1) & 1, wc)) break;
-        if ((p.debug_flags & 1) && j == 0) break;   // test hook: never deliver block 0
-        mbar_arrive_expect_tx(&full[st], L::TILE);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(ring + st * L::TILE + c * L::SUB, map, &full[st], c * 64, j * 128, bh);
-        issued = j + 1;
-      }
       // every copy this thread started must land before the CTA releases its shared memory
-      if (is_k) mbar_drain(q_full, 0, p.wait_ns);
-      for (int j = max(0, issued - NS); j < issued; ++j) mbar_drain(&full[j % NS], (j / NS) & 1, p.wait_ns);
+      for (int j = max(0, g - NS); j < g; ++j) mbar_drain(&full[j % NS], (j / NS) & 1, p.wait_ns);
     }
     __syncwarp();
   } else if (warp == 9) {
     // =========================================================== MMA issuer
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
-    if (lane == 0 && n_max > 0) {
+    reg_dealloc();
+    if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
       constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
-      const int n_a = tile_n_kv(0), n_b = tile_n_kv(1);
-      auto issue_s = [&](int x, int j) {   // S_x(j) = Q_x K_j^T
-        const uint32_t q_base = smem_u32(smem + (x ? L::QB_OFF : L::QA_OFF));
-        const uint32_t k_base = smem_u32(smem + L::K_OFF + (j % KST) * L::TILE);
+      int gk = 0, gv = 0;        // K and V blocks consumed (all items)
+      int nb[2] = {0, 0};        // blocks of each tile so far: phase of s_full / p_full
+      int ni[2] = {0, 0};        // items with work for each tile so far: phase of o_fin / o_free
+      int n_q = 0;               // Q pairs consumed
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int k = fwd_snake(r, cta, G);
+        if (k >= n_items) break;
+        int pair, bh;
+        fwd_item(k, p.n_pairs, BH, pair, bh);
+        const int n_a = tile_n_kv(pair, bh, 0), n_b = tile_n_kv(pair, bh, 1);
+        const int n_max = max(n_a, n_b);
+        if (n_max == 0) continue;
+        int s_left = n_a + n_b;   // S MMAs of this item still to issue (Q stays busy until the last)
+        auto issue_s = [&](int x, int j) {   // S_x(j) = Q_x K_j^T
+          const uint32_t q_base = smem_u32(smem + (x ? L::QB_OFF : L::QA_OFF));
+          const uint32_t k_base = smem_u32(smem + L::K_OFF + ((gk + j) % KST) * L::TILE);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
-          const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
-          mma_ss(tmem + L::s_col(x), sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
-                 kIdS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&s_full[x]);
-      };
-      auto issue_pv_half = [&](int x, int j, int h) {   // O_x += P_x(j)[keys of half h] V_j[same keys]
-        const uint32_t v_base = smem_u32(smem + L::V_OFF + (j % VST) * L::TILE);
+          for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
+            const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
+            mma_ss(tmem + L::s_col(x), sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                   kIdS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_full[x]);
+          if (--s_left == 0) mma_commit(q_empty);   // the next item's Q tiles may load now
+        };
+        auto issue_pv_half = [&](int x, int j, int h) {   // O_x += P_x(j)[keys of half h] V_j[same keys]
+          const uint32_t v_base = smem_u32(smem + L::V_OFF + ((gv + j) % VST) * L::TILE);
 #pragma unroll
-        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
-          mma_ts(tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_sw128(v_base + kk * 2048, L::SUB, 1024),
-                 kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
-      if (ok) {
+          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
+            mma_ts(tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_sw128(v_base + kk * 2048, L::SUB, 1024),
+                   kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
+        };
+        if (!mbar_wait(q_full, n_q & 1, wc) || !mbar_wait(&k_full[gk % KST], (gk / KST) & 1, wc)) { ok = false; break; }
+        ++n_q;
         tc_fence_after();
         if (n_a > 0) issue_s(0, 0);
         if (n_b > 0) issue_s(1, 0);
-        mma_commit(&k_empty[0]);
-      }
-      for (int j = 0; ok && j < n_max; ++j) {
-        if (!mbar_wait(&v_full[j % VST], (j / VST) & 1, wc)) { ok = false; break; }
-        const bool more = j + 1 < n_max;
-        bool have_k = false;   // K_{j+1} resident
+        mma_commit(&k_empty[gk % KST]);
+        for (int j = 0; ok && j < n_max; ++j) {
+          if (!mbar_wait(&v_full[(gv + j) % VST], ((gv + j) / VST) & 1, wc)) { ok = false; break; }
+          bool have_k = false;   // K_{j+1} resident
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int n_x = x ? n_b : n_a;
-          if (j >= n_x) continue;
+          for (int x = 0; x < 2; ++x) {
+            const int n_x = x ? n_b : n_a;
+            if (j >= n_x) continue;
+            // the first PV of an item overwrites O: the previous item's epilogue must have read it
+            if (j == 0 && ni[x] >= 1 && !mbar_wait(&o_free[x], (ni[x] - 1) & 1, wc)) { ok = false; break; }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait(&p_full[2 * x + h], j & 1, wc)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv_half(x, j, h);
+            for (int h = 0; h < 2; ++h) {
+              if (!mbar_wait(&p_full[2 * x + h], (nb[x] + j) & 1, wc)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv_half(x, j, h);
+            }
+            if (!ok) break;
+            if (j + 1 < n_x) {
+              if (!have_k) {
+                if (!mbar_wait(&k_full[(gk + j + 1) % KST], ((gk + j + 1) / KST) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                have_k = true;
+              }
+              issue_s(x, j + 1);
+            } else {
+              mma_commit(&o_fin[x]);
+            }
           }
           if (!ok) break;
-          if (j + 1 < n_x) {
-            if (!have_k) {
-              if (!mbar_wait(&k_full[(j + 1) % KST], ((j + 1) / KST) & 1, wc)) { ok = false; break; }
-              tc_fence_after();
-              have_k = true;
-            }
-            issue_s(x, j + 1);
-          } else {
-            mma_commit(&o_fin[x]);
-          }
+          mma_commit(&v_empty[(gv + j) % VST]);                       // V_j: both tiles' PV issued
+          if (j + 1 < n_max) mma_commit(&k_empty[(gk + j + 1) % KST]);  // K_{j+1}: both tiles' S issued
         }
-        if (!ok) break;
-        mma_commit(&v_empty[j % VST]);                  // V_j: both tiles' PV issued
-        if (more) mma_commit(&k_empty[(j + 1) % KST]);  // K_{j+1}: both tiles' S issued
+        gk += n_max;
+        gv += n_max;
+        nb[0] += n_a;
+        nb[1] += n_b;
+        ni[0] += (n_a > 0);
+        ni[1] += (n_b > 0);
       }
       mma_commit(fin);   // completes when every MMA issued above has finished
       mbar_drain(fin, 0, p.wait_ns);
@@ -255,130 +322,145 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else {
     // =========================================================== softmax / epilogue (warps 0-7)
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
+    reg_alloc();
     const int x = warp >> 2;   // tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int q0x = tile_q0(x);
-    const int q_row = q0x + r;
-    const int n = tile_n_kv(x);
-    const int kv_x = tile_kv_end(x);
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const uint32_t s_addr = lane_base + L::s_col(x);
     const uint32_t o_addr = lane_base + L::o_col(x);
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_make(sl2, sl2);
-    const uint64_t drop_row = (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * uint64_t(p.N);
-    float m_ref = -INFINITY;   // reference max, exp2 domain
-    float l = 0.f;
+    int nb = 0, ni = 0;   // blocks and items of this tile so far (barrier phases)
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, wc))) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      tmem_ld_wait();
+    for (int rr = 0; ok; ++rr) {
+      const int k = fwd_snake(rr, cta, G);
+      if (k >= n_items) break;
+      int pair, bh;
+      fwd_item(k, p.n_pairs, BH, pair, bh);
+      const int q0x = tile_q0(pair, x);
+      const int q_row = q0x + r;
+      const int n = tile_n_kv(pair, bh, x);
+      const int kv_x = tile_kv_end(pair, bh, x);
+      const uint64_t drop_row = (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * uint64_t(p.N);
+      float m_ref = -INFINITY;   // reference max, exp2 domain
+      float l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[x], (nb + j) & 1, wc))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_ld_wait();
 #pragma unroll
-      for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
+        for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
 
-      const int k0 = j * 128;
-      const bool masked = (k0 + 128 > kv_x) || (p.causal && k0 + 128 > q0x);   // block straddles a mask edge
-      if (masked) {
-        const int lim = min(kv_x, p.causal ? q_row + 1 : kv_x) - k0;   // columns < lim are kept
+        const int k0 = j * 128;
+        if ((k0 + 128 > kv_x) || (p.causal && k0 + 128 > q0x)) {   // block straddles a mask edge
+          const int lim = min(kv_x, p.causal ? q_row + 1 : kv_x) - k0;   // columns < lim are kept
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
-      }
-      float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
-#pragma unroll
-      for (int c = 0; c < 128; c += 8)
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          mxv[u] = max3f(mxv[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
-      const float mx = fmaxf(max3f(mxv[0], mxv[1], mxv[2]), mxv[3]);
-      const float m_cand = mx * sl2;
-      float alpha = 1.f;
-      if (m_cand > m_ref + kRescaleThreshold) {
-        alpha = ex2_approx(m_ref - m_cand);
-        m_ref = m_cand;
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const uint64_t negm2 = f2_make(-m_use, -m_use);
-      uint64_t rs2 = f2_make(0.f, 0.f);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {   // two halves of 64 keys; the MMA takes each half as soon as it is ready
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = 32 * h + e;   // pair index: keys 2c, 2c+1
-          const uint64_t pp = exp2_pair(sr[2 * c], sr[2 * c + 1], sl2x2, negm2);
-          rs2 = f2_add(rs2, pp);
-          float p0, p1;
-          f2_split(pp, p0, p1);
-          if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
-            const uint64_t ctr = drop_row + uint64_t(k0 + 2 * c);
-            p0 = dropout_keep(p.seed, ctr, p.drop_thr) ? p0 : 0.f;
-            p1 = dropout_keep(p.seed, ctr + 1, p.drop_thr) ? p1 : 0.f;
-          }
-          pk[e] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
-        // P over the score columns already read; O already holds PV up to block j-1
-        tmem_st32(s_addr + 32 * h, pk);
-        if (h == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(o_addr + c * 32, orr);
-            tmem_ld_wait();
-            reg_fence32(orr);
+        for (int c = 0; c < 128; c += 8)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-            tmem_st32(o_addr + c * 32, orr);
-          }
+          for (int u = 0; u < 4; ++u)
+            mxv[u] = max3f(mxv[u], __uint_as_float(sr[c + 2 * u]), __uint_as_float(sr[c + 2 * u + 1]));
+        const float mx = fmaxf(max3f(mxv[0], mxv[1], mxv[2]), mxv[3]);
+        const float m_cand = mx * sl2;
+        float alpha = 1.f;
+        if (m_cand > m_ref + kRescaleThreshold) {
+          alpha = ex2_approx(m_ref - m_cand);
+          m_ref = m_cand;
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[2 * x + h]);
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t negm2 = f2_make(-m_use, -m_use);
+        uint64_t rs2 = f2_make(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {   // two halves of 64 keys; the MMA takes each half as soon as it is ready
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c = 32 * h + e;   // pair index: keys 2c, 2c+1
+            const uint64_t pp = exp2_pair(sr[2 * c], sr[2 * c + 1], sl2x2, negm2);
+            rs2 = f2_add(rs2, pp);
+            float p0, p1;
+            f2_split(pp, p0, p1);
+            if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
+              const uint64_t ctr = drop_row + uint64_t(k0 + 2 * c);
+              p0 = dropout_keep(p.seed, ctr, p.drop_thr) ? p0 : 0.f;
+              p1 = dropout_keep(p.seed, ctr + 1, p.drop_thr) ? p1 : 0.f;
+            }
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          // P over the score columns already read; O already holds PV up to block j-1
+          tmem_st32(s_addr + 32 * h, pk);
+          if (h == 0 && j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(o_addr + c * 32, orr);
+              tmem_ld_wait();
+              reg_fence32(orr);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+              tmem_st32(o_addr + c * 32, orr);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[2 * x + h]);
+        }
+        float rs0, rs1;
+        f2_split(rs2, rs0, rs1);
+        l = l * alpha + (rs0 + rs1);
       }
-      float rs0, rs1;
-      f2_split(rs2, rs0, rs1);
-      l = l * alpha + (rs0 + rs1);
-    }
+      if (!ok) break;
 
-    // ---- epilogue: O / l -> bf16, lse = (m + log2 l) * ln 2
-    const bool row_valid = q_row < p.N;
-    __nv_bfloat16* orow = p.o + (uint64_t(bh) * uint64_t(p.N) + uint64_t(row_valid ? q_row : 0)) * D;
-    if (n == 0) {
-      if (row_valid) {
+      // ---- epilogue: O / l -> bf16, lse = (m + log2 l) * ln 2
+      const bool row_valid = q_row < p.N;
+      __nv_bfloat16* orow = p.o + (uint64_t(bh) * uint64_t(p.N) + uint64_t(row_valid ? q_row : 0)) * D;
+      if (n == 0) {
+        if (row_valid) {
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
-        p.lse[uint64_t(bh) * p.N + q_row] = -INFINITY;
+          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = make_uint4(0, 0, 0, 0);
+          p.lse[uint64_t(bh) * p.N + q_row] = -INFINITY;
+        }
+        continue;
       }
-    } else if (ok && __all_sync(0xffffffffu, mbar_wait(&o_fin[x], 0, wc))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_fin[x], ni & 1, wc))) { ok = false; break; }
       tc_fence_after();
       const float inv_l = l > 0.f ? (DROPOUT ? p.drop_scale : 1.f) / l : 0.f;
+      uint32_t packed[D / 2];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
         tmem_ld32(o_addr + c * 32, orr);
         tmem_ld_wait();
         reg_fence32(orr);
-        uint32_t packed[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          packed[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-        }
+          packed[16 * c + e] =
+              pack_bf16x2(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
       }
-      if (row_valid) p.lse[uint64_t(bh) * p.N + q_row] = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : -INFINITY;
+      // O is in registers: the next item's first PV may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[x]);
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+        for (int e = 0; e < D / 8; ++e)
+          dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        p.lse[uint64_t(bh) * p.N + q_row] = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : -INFINITY;
+      }
+      nb += n;
+      ++ni;
     }
   }
 
