@@ -7,8 +7,8 @@
 // blocks and both tiles share every K/V block.  The grid is persistent (one CTA per SM): each CTA
 // takes the items of a heavy-first list in snake order (round r: CTA c takes item r*G + c, or
 // r*G + G-1-c on odd rounds), and its pipelines run on from one item into the next: the K/V rings
-// continue, the next Q tiles load as soon as the last S of an item has been issued, and the next
-// item's first S overlaps the epilogue of the previous one.  Warp roles (three warpgroups):
+// continue, each next Q tile loads as soon as the last S of its tile has been issued, and the
+// next item's first S overlaps the epilogue of the previous one.  Warp roles (three warpgroups):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns query row r of its
 //              tile (= TMEM lane r); masks, exponentiates, writes P (bf16) over the tile's score
 //              columns, rescales O when needed, writes O and lse at the end
@@ -64,9 +64,9 @@ struct FwdLayout {
   static constexpr int K_OFF = QB_OFF + TILE;
   static constexpr int V_OFF = K_OFF + KST * TILE;
   static constexpr int BAR_OFF = V_OFF + VST * TILE;
-  // q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], p_full[2][2],
-  // o_fin[2], o_free[2], fin
-  static constexpr int NBARS = 2 + 2 * KST + 2 * VST + 2 + 4 + 2 + 2 + 1;
+  // q_full[2], q_empty[2], k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
+  // p_full[2][2], o_fin[2], o_free[2], fin
+  static constexpr int NBARS = 4 + 2 * KST + 2 * VST + 2 + 4 + 2 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   __device__ static constexpr int s_col(int x) { return 128 * x; }         // S_A, S_B
@@ -108,9 +108,9 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = q_full + 1;
-  uint64_t* k_full = q_empty + 1;
+  uint64_t* q_full = bars;           // [2]: tile A, tile B
+  uint64_t* q_empty = q_full + 2;    // [2]
+  uint64_t* k_full = q_empty + 2;
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + VST;
@@ -141,8 +141,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   };
 
   if (tid == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+    }
     for (int s = 0; s < KST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -180,24 +182,29 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     reg_dealloc();
     if (lane == 0) {
       prefetch_tmap(&tm_q);
-      int n_q = 0;          // Q pairs delivered
-      for (int r = 0;; ++r) {
+      int nq[2] = {0, 0};   // Q tiles delivered, per tile
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
         const int k = fwd_snake(r, cta, G);
         if (k >= n_items) break;
         int pair, bh;
         fwd_item(k, p.n_pairs, BH, pair, bh);
-        if (max(tile_n_kv(pair, bh, 0), tile_n_kv(pair, bh, 1)) == 0) continue;
-        // both Q tiles, once the previous item's last S has read the buffers
-        if (n_q >= 1 && !mbar_wait(q_empty, (n_q - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(q_full, 2 * L::TILE);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + L::QA_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(pair, 0), bh);
-          tma_load_3d(smem + L::QB_OFF + c * L::SUB, &tm_q, q_full, c * 64, tile_q0(pair, 1), bh);
+        for (int x = 0; x < 2; ++x) {
+          if (tile_n_kv(pair, bh, x) == 0) continue;
+          // tile x of this item, once the previous item's last S of tile x has read the buffer
+          if (nq[x] >= 1 && !mbar_wait(&q_empty[x], (nq[x] - 1) & 1, wc)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[x], L::TILE);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem + (x ? L::QB_OFF : L::QA_OFF) + c * L::SUB, &tm_q, &q_full[x], c * 64,
+                        tile_q0(pair, x), bh);
+          ++nq[x];
         }
-        ++n_q;
       }
-      if (n_q >= 1) mbar_drain(q_full, (n_q - 1) & 1, p.wait_ns);   // the last copies land before exit
+#pragma unroll
+      for (int x = 0; x < 2; ++x)   // the last copies land before the CTA exits
+        if (nq[x] >= 1) mbar_drain(&q_full[x], (nq[x] - 1) & 1, p.wait_ns);
     }
     __syncwarp();
   } else if (warp == 8 || warp == 10) {
@@ -242,7 +249,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       int gk = 0, gv = 0;        // K and V blocks consumed (all items)
       int nb[2] = {0, 0};        // blocks of each tile so far: phase of s_full / p_full
       int ni[2] = {0, 0};        // items with work for each tile so far: phase of o_fin / o_free
-      int n_q = 0;               // Q pairs consumed
+      int nq[2] = {0, 0};        // Q tiles consumed, per tile
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int k = fwd_snake(r, cta, G);
@@ -252,7 +259,6 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int n_a = tile_n_kv(pair, bh, 0), n_b = tile_n_kv(pair, bh, 1);
         const int n_max = max(n_a, n_b);
         if (n_max == 0) continue;
-        int s_left = n_a + n_b;   // S MMAs of this item still to issue (Q stays busy until the last)
         auto issue_s = [&](int x, int j) {   // S_x(j) = Q_x K_j^T
           const uint32_t q_base = smem_u32(smem + (x ? L::QB_OFF : L::QA_OFF));
           const uint32_t k_base = smem_u32(smem + L::K_OFF + ((gk + j) % KST) * L::TILE);
@@ -263,7 +269,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                    kIdS, kk > 0 ? 1u : 0u);
           }
           mma_commit(&s_full[x]);
-          if (--s_left == 0) mma_commit(q_empty);   // the next item's Q tiles may load now
+          if (j + 1 == (x ? n_b : n_a)) mma_commit(&q_empty[x]);   // the next item's Q_x may load now
         };
         auto issue_pv_half = [&](int x, int j, int h) {   // O_x += P_x(j)[keys of half h] V_j[same keys]
           const uint32_t v_base = smem_u32(smem + L::V_OFF + ((gv + j) % VST) * L::TILE);
@@ -272,11 +278,16 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mma_ts(tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_sw128(v_base + kk * 2048, L::SUB, 1024),
                    kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
         };
-        if (!mbar_wait(q_full, n_q & 1, wc) || !mbar_wait(&k_full[gk % KST], (gk / KST) & 1, wc)) { ok = false; break; }
-        ++n_q;
-        tc_fence_after();
-        if (n_a > 0) issue_s(0, 0);
-        if (n_b > 0) issue_s(1, 0);
+        if (!mbar_wait(&k_full[gk % KST], (gk / KST) & 1, wc)) { ok = false; break; }
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if ((x ? n_b : n_a) == 0) continue;
+          if (!mbar_wait(&q_full[x], nq[x] & 1, wc)) { ok = false; break; }
+          ++nq[x];
+          tc_fence_after();
+          issue_s(x, 0);
+        }
+        if (!ok) break;
         mma_commit(&k_empty[gk % KST]);
         for (int j = 0; ok && j < n_max; ++j) {
           if (!mbar_wait(&v_full[(gv + j) % VST], ((gv + j) / VST) & 1, wc)) { ok = false; break; }
