@@ -59,6 +59,7 @@ struct BwdParams {  // (the main kernel also takes tensor maps of q, k, v, dO an
   float drop_scale;
   uint64_t seed;
   uint64_t wait_ns;
+  int out_align32;             // dk and dv are 32-byte aligned: epilogues use 32-byte stores
 };
 
 constexpr float kLog2e = 1.4426950408889634074f;
@@ -140,6 +141,22 @@ struct BwdLayout {
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
+
+// 32 fp32 values of one row, scaled and rounded to bf16, stored as 64 bytes (two 32-byte stores
+// when the destination allows it, else four 16-byte stores).
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&v)[32], float s, int align32) {
+  uint32_t w[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * s, __uint_as_float(v[2 * e + 1]) * s);
+  if (align32) {
+    st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    st_global_v8(dst + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+  }
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, w));
@@ -522,15 +539,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_ld32(lane_base + L::DV_COL + c * 32, vr);
         tmem_ld_wait();
         reg_fence32(vr);
-        if (key < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dv + (row_base + key) * D + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(vr[8 * e]) * s, __uint_as_float(vr[8 * e + 1]) * s),
-                                pack_bf16x2(__uint_as_float(vr[8 * e + 2]) * s, __uint_as_float(vr[8 * e + 3]) * s),
-                                pack_bf16x2(__uint_as_float(vr[8 * e + 4]) * s, __uint_as_float(vr[8 * e + 5]) * s),
-                                pack_bf16x2(__uint_as_float(vr[8 * e + 6]) * s, __uint_as_float(vr[8 * e + 7]) * s));
-        }
+        if (key < p.N) store_row32(p.dv + (row_base + key) * D + c * 32, vr, s, p.out_align32);
       }
     }
   } else {
@@ -595,15 +604,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_ld32(lane_base + L::DK_COL + c * 32, kr);
         tmem_ld_wait();
         reg_fence32(kr);
-        if (key < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(p.dk + (row_base + key) * D + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pack_bf16x2(__uint_as_float(kr[8 * e]) * s, __uint_as_float(kr[8 * e + 1]) * s),
-                                pack_bf16x2(__uint_as_float(kr[8 * e + 2]) * s, __uint_as_float(kr[8 * e + 3]) * s),
-                                pack_bf16x2(__uint_as_float(kr[8 * e + 4]) * s, __uint_as_float(kr[8 * e + 5]) * s),
-                                pack_bf16x2(__uint_as_float(kr[8 * e + 6]) * s, __uint_as_float(kr[8 * e + 7]) * s));
-        }
+        if (key < p.N) store_row32(p.dk + (row_base + key) * D + c * 32, kr, s, p.out_align32);
       }
     }
   }

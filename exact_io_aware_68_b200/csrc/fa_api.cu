@@ -248,6 +248,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.seed = seed;
   p.wait_ns = g_wait_ns.load();
   p.debug_flags = g_debug_flags.load();
+  p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64) return p.dropout ? launch_fwd<64, true>(mq, mk, mv, p, s) : launch_fwd<64, false>(mq, mk, mv, p, s);
   return p.dropout ? launch_fwd<128, true>(mq, mk, mv, p, s) : launch_fwd<128, false>(mq, mk, mv, p, s);
@@ -336,6 +337,7 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* 
   p.lse = lse;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.out_align32 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, p, s)

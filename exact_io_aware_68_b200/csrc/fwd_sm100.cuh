@@ -48,6 +48,7 @@ struct FwdParams {
   uint64_t seed;
   uint64_t wait_ns;
   int debug_flags;             // bit 0: producer skips the first K/V load (exercises the timeout path)
+  int o_align32;               // o is 32-byte aligned: the epilogue uses 32-byte stores
 };
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 domain
@@ -464,10 +465,17 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[x]);
       if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow);
+        if (p.o_align32) {
 #pragma unroll
-        for (int e = 0; e < D / 8; ++e)
-          dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+          for (int e = 0; e < D / 16; ++e)
+            st_global_v8(orow + 16 * e, packed[8 * e], packed[8 * e + 1], packed[8 * e + 2], packed[8 * e + 3],
+                         packed[8 * e + 4], packed[8 * e + 5], packed[8 * e + 6], packed[8 * e + 7]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int e = 0; e < D / 8; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
         p.lse[uint64_t(bh) * p.N + q_row] = l > 0.f ? (m_ref + lg2_approx(l)) * kLn2 : -INFINITY;
       }
       nb += n;

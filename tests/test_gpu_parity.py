@@ -145,3 +145,22 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     *_, o, lse = run_fwd(x)
     O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"])
     assert_o_close(to_f64(o), O, O_MAX_ABS_BF16)
+
+
+def test_outputs_only_16_byte_aligned():
+    """Outputs that are 16- but not 32-byte aligned take the 16-byte store path of the epilogues."""
+    w = wl(2, 2, 200, 128, causal=True, seed=31)
+    x = make_inputs(w)
+    q, k, v, do = (to_device(x, n) for n in ("q", "k", "v", "do"))
+    n = q.numel()
+    bufs = [torch.empty(n + 8, dtype=torch.bfloat16, device="cuda") for _ in range(4)]   # 8 bf16 = 16 bytes
+    o, dq, dk, dv = (b[8:8 + n].view(q.shape) for b in bufs)
+    assert all(t.data_ptr() % 32 == 16 for t in (o, dq, dk, dv))
+    o, lse = api.attention_fwd(q, k, v, w.scale, True, o=o)
+    api.attention_bwd(q, k, v, o, lse, do, w.scale, True, dq=dq, dk=dk, dv=dv)
+    api.check()
+    O, L = oracle.forward(x["q64"], x["k64"], x["v64"], w.scale, True)
+    assert_o_close(to_f64(o), O, O_MAX_ABS_BF16)
+    ref = oracle.backward(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, True)
+    for g, r in zip((dq, dk, dv), ref):
+        assert rel_l2(to_f64(g), r) <= GRAD_REL_L2
