@@ -243,94 +243,102 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp == 9) {
     // =========================================================== MMA issuer
+    // The whole warp runs the loop (descriptors stay warp-uniform); lane 0 issues every MMA and
+    // commit, so one thread owns all tcgen05 work and each commit covers every MMA before it.
     reg_dealloc();
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
-      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
-      int gk = 0, gv = 0;        // K and V blocks consumed (all items)
-      int nb[2] = {0, 0};        // blocks of each tile so far: phase of s_full / p_full
-      int ni[2] = {0, 0};        // items with work for each tile so far: phase of o_fin / o_free
-      int nq[2] = {0, 0};        // Q tiles consumed, per tile
-      bool ok = true;
-      for (int r = 0; ok; ++r) {
-        const int k = fwd_snake(r, cta, G);
-        if (k >= n_items) break;
-        int pair, bh;
-        fwd_item(k, p.n_pairs, BH, pair, bh);
-        const int n_a = tile_n_kv(pair, bh, 0), n_b = tile_n_kv(pair, bh, 1);
-        const int n_max = max(n_a, n_b);
-        if (n_max == 0) continue;
-        auto issue_s = [&](int x, int j) {   // S_x(j) = Q_x K_j^T
-          const uint32_t q_base = smem_u32(smem + (x ? L::QB_OFF : L::QA_OFF));
-          const uint32_t k_base = smem_u32(smem + L::K_OFF + ((gk + j) % KST) * L::TILE);
+    const uint32_t lead = lane == 0 ? 1u : 0u;
+    auto wait = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc)); };
+    constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
+    constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
+    // descriptor of each buffer's first byte; a byte offset `o` inside it is desc + (o >> 4)
+    const uint64_t qdesc[2] = {sdesc_sw128(smem_u32(smem + L::QA_OFF), 16, 1024),
+                               sdesc_sw128(smem_u32(smem + L::QB_OFF), 16, 1024)};
+    const uint64_t kdesc = sdesc_sw128(smem_u32(smem + L::K_OFF), 16, 1024);
+    const uint64_t vdesc = sdesc_sw128(smem_u32(smem + L::V_OFF), L::SUB, 1024);
+    int gk = 0, gv = 0;        // K and V blocks consumed (all items)
+    int nb[2] = {0, 0};        // blocks of each tile so far: phase of s_full / p_full
+    int ni[2] = {0, 0};        // items with work for each tile so far: phase of o_fin / o_free
+    int nq[2] = {0, 0};        // Q tiles consumed, per tile
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int k = fwd_snake(r, cta, G);
+      if (k >= n_items) break;
+      int pair, bh;
+      fwd_item(k, p.n_pairs, BH, pair, bh);
+      const int n_a = tile_n_kv(pair, bh, 0), n_b = tile_n_kv(pair, bh, 1);
+      const int n_max = max(n_a, n_b);
+      if (n_max == 0) continue;
+      auto issue_s = [&](int x, int kst) {   // S_x = Q_x K^T, K in ring stage kst
+        const uint64_t kd = kdesc + uint32_t(kst * (L::TILE >> 4));
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
-            const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
-            mma_ss(tmem + L::s_col(x), sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
-                   kIdS, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&s_full[x]);
-          if (j + 1 == (x ? n_b : n_a)) mma_commit(&q_empty[x]);   // the next item's Q_x may load now
-        };
-        auto issue_pv_half = [&](int x, int j, int h) {   // O_x += P_x(j)[keys of half h] V_j[same keys]
-          const uint32_t v_base = smem_u32(smem + L::V_OFF + ((gv + j) % VST) * L::TILE);
+        for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
+          const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
+          mma_ss_lead(lead, tmem + L::s_col(x), qdesc[x] + off, kd + off, kIdS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv_half = [&](int x, int vst, int h, uint32_t acc0) {   // O_x += P_x[keys of half h] V[same keys]
+        const uint64_t vd = vdesc + uint32_t(vst * (L::TILE >> 4));
 #pragma unroll
-          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
-            mma_ts(tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_sw128(v_base + kk * 2048, L::SUB, 1024),
-                   kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
-        };
-        if (!mbar_wait(&k_full[gk % KST], (gk / KST) & 1, wc)) { ok = false; break; }
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
+          mma_ts_lead(lead, tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, vd + uint32_t(kk * (2048 >> 4)), kIdPV,
+                      kk > 0 ? 1u : acc0);
+      };
+      if (!wait(&k_full[gk % KST], (gk / KST) & 1)) { ok = false; break; }
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if ((x ? n_b : n_a) == 0) continue;
+        if (!wait(&q_full[x], nq[x] & 1)) { ok = false; break; }
+        ++nq[x];
+        tc_fence_after();
+        issue_s(x, gk % KST);
+        mma_commit_lead(lead, &s_full[x]);
+        if (1 == (x ? n_b : n_a)) mma_commit_lead(lead, &q_empty[x]);   // the next item's Q_x may load now
+      }
+      if (!ok) break;
+      mma_commit_lead(lead, &k_empty[gk % KST]);
+      for (int j = 0; ok && j < n_max; ++j) {
+        const int vst = (gv + j) % VST, kst1 = (gk + j + 1) % KST;
+        if (!wait(&v_full[vst], ((gv + j) / VST) & 1)) { ok = false; break; }
+        bool have_k = false;   // K_{j+1} resident
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          if ((x ? n_b : n_a) == 0) continue;
-          if (!mbar_wait(&q_full[x], nq[x] & 1, wc)) { ok = false; break; }
-          ++nq[x];
-          tc_fence_after();
-          issue_s(x, 0);
-        }
-        if (!ok) break;
-        mma_commit(&k_empty[gk % KST]);
-        for (int j = 0; ok && j < n_max; ++j) {
-          if (!mbar_wait(&v_full[(gv + j) % VST], ((gv + j) / VST) & 1, wc)) { ok = false; break; }
-          bool have_k = false;   // K_{j+1} resident
+          const int n_x = x ? n_b : n_a;
+          if (j >= n_x) continue;
+          // the first PV of an item overwrites O: the previous item's epilogue must have read it
+          if (j == 0 && ni[x] >= 1 && !wait(&o_free[x], (ni[x] - 1) & 1)) { ok = false; break; }
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const int n_x = x ? n_b : n_a;
-            if (j >= n_x) continue;
-            // the first PV of an item overwrites O: the previous item's epilogue must have read it
-            if (j == 0 && ni[x] >= 1 && !mbar_wait(&o_free[x], (ni[x] - 1) & 1, wc)) { ok = false; break; }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (!mbar_wait(&p_full[2 * x + h], (nb[x] + j) & 1, wc)) { ok = false; break; }
-              tc_fence_after();
-              issue_pv_half(x, j, h);
-            }
-            if (!ok) break;
-            if (j + 1 < n_x) {
-              if (!have_k) {
-                if (!mbar_wait(&k_full[(gk + j + 1) % KST], ((gk + j + 1) / KST) & 1, wc)) { ok = false; break; }
-                tc_fence_after();
-                have_k = true;
-              }
-              issue_s(x, j + 1);
-            } else {
-              mma_commit(&o_fin[x]);
-            }
+          for (int h = 0; h < 2; ++h) {
+            if (!wait(&p_full[2 * x + h], (nb[x] + j) & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv_half(x, vst, h, j > 0 ? 1u : 0u);
           }
           if (!ok) break;
-          mma_commit(&v_empty[(gv + j) % VST]);                       // V_j: both tiles' PV issued
-          if (j + 1 < n_max) mma_commit(&k_empty[(gk + j + 1) % KST]);  // K_{j+1}: both tiles' S issued
+          if (j + 1 < n_x) {
+            if (!have_k) {
+              if (!wait(&k_full[kst1], ((gk + j + 1) / KST) & 1)) { ok = false; break; }
+              tc_fence_after();
+              have_k = true;
+            }
+            issue_s(x, kst1);
+            mma_commit_lead(lead, &s_full[x]);
+            if (j + 2 == n_x) mma_commit_lead(lead, &q_empty[x]);   // the next item's Q_x may load now
+          } else {
+            mma_commit_lead(lead, &o_fin[x]);
+          }
         }
-        gk += n_max;
-        gv += n_max;
-        nb[0] += n_a;
-        nb[1] += n_b;
-        ni[0] += (n_a > 0);
-        ni[1] += (n_b > 0);
+        if (!ok) break;
+        mma_commit_lead(lead, &v_empty[vst]);                       // V_j: both tiles' PV issued
+        if (j + 1 < n_max) mma_commit_lead(lead, &k_empty[kst1]);   // K_{j+1}: both tiles' S issued
       }
-      mma_commit(fin);   // completes when every MMA issued above has finished
-      mbar_drain(fin, 0, p.wait_ns);
+      gk += n_max;
+      gv += n_max;
+      nb[0] += n_a;
+      nb[1] += n_b;
+      ni[0] += (n_a > 0);
+      ni[1] += (n_b > 0);
     }
+    mma_commit_lead(lead, fin);   // completes when every MMA issued above has finished
+    if (lead) mbar_drain(fin, 0, p.wait_ns);
     __syncwarp();
   } else {
     // =========================================================== softmax / epilogue (warps 0-7)
