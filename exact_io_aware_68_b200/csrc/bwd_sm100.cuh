@@ -323,41 +323,44 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp == 9) {
     // =========================================================== MMA issuer
+    // The whole warp runs the loop (descriptors stay warp-uniform); lane 0 issues every MMA and
+    // commit under a predicate, so one thread owns all tcgen05 work.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
-    if (lane == 0 && n_iter > 0) {
+    const uint32_t lead = lane == 0 ? 1u : 0u;
+    if (n_iter > 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (V) and Q (dO) K-major
       constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A K-major, B MN-major
       constexpr uint32_t kIdQ = idesc_bf16(D, 128, true, true);       // dQ^T: K^T, dS^T both MN-major
-      const uint32_t k_base = smem_u32(smem + L::K_OFF);
-      const uint32_t v_base = smem_u32(smem + L::V_OFF);
-      const uint32_t ds_base = smem_u32(smem + L::DS_OFF);
-      auto q_at = [&](int t) { return smem_u32(smem + L::Q_OFF + (t % QS) * L::TILE); };
-      auto do_at = [&](int t) { return smem_u32(smem + L::DO_OFF + (t % DS) * L::TILE); };
+      // descriptors: low word = s0 + (byte offset in shared memory >> 4) + leading-offset field
+      // (K-major: 16; MN-major: one 64-column panel)
+      const uint32_t s0 = smem_u32(smem) >> 4;
+      constexpr uint32_t kHi = sdesc_sw128_hi(1024), kKM = sdesc_lbo(16), kMN = sdesc_lbo(L::SUB);
+      auto lo = [&](int off, uint32_t lbo) { return s0 + uint32_t(off >> 4) + lbo; };
       auto issue_s = [&](int t) {   // S^T = K Q_t^T  (M = 128 keys, N = 128 queries, K = D)
-        const uint32_t q_base = q_at(t);
+        const uint32_t k_lo = lo(L::K_OFF, kKM), q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kKM);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
-          mma_ss(tmem + L::ST_COL, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(q_base + off, 16, 1024), kIdS,
-                 kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
+          mma_ss_lead(lead, tmem + L::ST_COL, sdesc_join(k_lo + off, kHi), sdesc_join(q_lo + off, kHi), kIdS,
+                      kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full);
+        mma_commit_lead(lead, s_full);
       };
       auto issue_dp = [&](int t) {   // dP^T = V dO_t^T
-        const uint32_t do_base = do_at(t);
+        const uint32_t v_lo = lo(L::V_OFF, kKM), do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kKM);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::SUB + (kk & 3) * 32;
-          mma_ss(tmem + L::DPT_COL, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(do_base + off, 16, 1024),
-                 kIdS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
+          mma_ss_lead(lead, tmem + L::DPT_COL, sdesc_join(v_lo + off, kHi), sdesc_join(do_lo + off, kHi), kIdS,
+                      kk > 0 ? 1u : 0u);
         }
-        mma_commit(dp_full);
+        mma_commit_lead(lead, dp_full);
       };
-      bool ok = mbar_wait(kv_full, 0, wc) && mbar_wait(&q_full[0], 0, wc);
+      bool ok = warp_wait(kv_full, 0, wc) && warp_wait(&q_full[0], 0, wc);
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        ok = mbar_wait(&do_full[0], 0, wc);
+        ok = warp_wait(&do_full[0], 0, wc);
         if (ok) {
           tc_fence_after();
           issue_dp(0);
@@ -365,45 +368,55 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       for (int t = 0; ok && t < n_iter; ++t) {
         const bool more = t + 1 < n_iter;
+        const uint32_t acc0 = t > 0 ? 1u : 0u;
         // dV += (P*Z)^T dO_t   (A = (P*Z)^T in TMEM, B = dO MN-major: N = D, K = queries)
-        if (!mbar_wait(p_full, t & 1, wc)) { ok = false; break; }
+        if (!warp_wait(p_full, t & 1, wc)) { ok = false; break; }
         tc_fence_after();
+        {
+          const uint32_t do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kMN);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_sw128(do_at(t) + kk * 2048, L::SUB, 1024), kIdG,
-                 (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&do_empty[t % DS]);   // dO_t: last read by dV_t
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_lead(lead, tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_join(do_lo + kk * (2048 >> 4), kHi),
+                        kIdG, kk > 0 ? 1u : acc0);
+        }
+        mma_commit_lead(lead, &do_empty[t % DS]);   // dO_t: last read by dV_t
         // S_{t+1} over the (P*Z)^T that dV_t has just been given (MMAs run in issue order)
         if (more) {
-          if (!mbar_wait(&q_full[(t + 1) % QS], ((t + 1) / QS) & 1, wc)) { ok = false; break; }
+          if (!warp_wait(&q_full[(t + 1) % QS], ((t + 1) / QS) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           issue_s(t + 1);
         }
         // dQ^T = K^T dS^T into the dP^T columns (already read)   (M = D, N = 128 queries, K = 128 keys)
-        if (!mbar_wait(ds_full, t & 1, wc)) { ok = false; break; }
+        if (!warp_wait(ds_full, t & 1, wc)) { ok = false; break; }
         tc_fence_after();
+        {
+          const uint32_t k_lo = lo(L::K_OFF, kMN), ds_lo = lo(L::DS_OFF, kMN);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::DPT_COL, sdesc_sw128(k_base + kk * 2048, L::SUB, 1024),
-                 sdesc_sw128(ds_base + kk * 2048, L::SUB, 1024), kIdQ, kk > 0 ? 1u : 0u);
-        mma_commit(dq_full);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss_lead(lead, tmem + L::DPT_COL, sdesc_join(k_lo + kk * (2048 >> 4), kHi),
+                        sdesc_join(ds_lo + kk * (2048 >> 4), kHi), kIdQ, kk > 0 ? 1u : 0u);
+        }
+        mma_commit_lead(lead, dq_full);
         // dK += dS^T Q_t   (A = dS^T from shared memory, K-major: rows = keys, 16 queries per step)
+        {
+          const uint32_t ds_lo = lo(L::DS_OFF, kKM), q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kMN);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::DK_COL, sdesc_sw128(ds_base + (kk >> 2) * L::SUB + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(q_at(t) + kk * 2048, L::SUB, 1024), kIdG, (t > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(dk_done);             // the dS tile is free again
-        mma_commit(&q_empty[t % QS]);    // Q_t: last read by dK_t
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss_lead(lead, tmem + L::DK_COL, sdesc_join(ds_lo + (((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4), kHi),
+                        sdesc_join(q_lo + kk * (2048 >> 4), kHi), kIdG, kk > 0 ? 1u : acc0);
+        }
+        mma_commit_lead(lead, dk_done);             // the dS tile is free again
+        mma_commit_lead(lead, &q_empty[t % QS]);    // Q_t: last read by dK_t
         // dP_{t+1} once the dQ warps have read dQ^T out of those columns
         if (more) {
-          if (!mbar_wait(dq_empty, t & 1, wc)) { ok = false; break; }
-          if (!mbar_wait(&do_full[(t + 1) % DS], ((t + 1) / DS) & 1, wc)) { ok = false; break; }
+          if (!warp_wait(dq_empty, t & 1, wc)) { ok = false; break; }
+          if (!warp_wait(&do_full[(t + 1) % DS], ((t + 1) / DS) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           issue_dp(t + 1);
         }
       }
-      mma_commit(fin);
-      mbar_drain(fin, 0, p.wait_ns);
+      mma_commit_lead(lead, fin);
+      if (lead) mbar_drain(fin, 0, p.wait_ns);
     }
     __syncwarp();
   } else if (warp < 4) {

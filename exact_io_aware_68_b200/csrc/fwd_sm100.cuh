@@ -250,11 +250,9 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto wait = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc)); };
     constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
     constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
-    // descriptor of each buffer's first byte; a byte offset `o` inside it is desc + (o >> 4)
-    const uint64_t qdesc[2] = {sdesc_sw128(smem_u32(smem + L::QA_OFF), 16, 1024),
-                               sdesc_sw128(smem_u32(smem + L::QB_OFF), 16, 1024)};
-    const uint64_t kdesc = sdesc_sw128(smem_u32(smem + L::K_OFF), 16, 1024);
-    const uint64_t vdesc = sdesc_sw128(smem_u32(smem + L::V_OFF), L::SUB, 1024);
+    // descriptors: low word = s0 + (byte offset in shared memory >> 4) + leading-offset field
+    const uint32_t s0 = smem_u32(smem) >> 4;
+    constexpr uint32_t kHi = sdesc_sw128_hi(1024), kKM = sdesc_lbo(16), kMN = sdesc_lbo(L::SUB);
     int gk = 0, gv = 0;        // K and V blocks consumed (all items)
     int nb[2] = {0, 0};        // blocks of each tile so far: phase of s_full / p_full
     int ni[2] = {0, 0};        // items with work for each tile so far: phase of o_fin / o_free
@@ -269,19 +267,21 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int n_max = max(n_a, n_b);
       if (n_max == 0) continue;
       auto issue_s = [&](int x, int kst) {   // S_x = Q_x K^T, K in ring stage kst
-        const uint64_t kd = kdesc + uint32_t(kst * (L::TILE >> 4));
+        const uint32_t q_lo = s0 + uint32_t((x ? L::QB_OFF : L::QA_OFF) >> 4) + kKM;
+        const uint32_t k_lo = s0 + uint32_t((L::K_OFF + kst * L::TILE) >> 4) + kKM;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
           const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
-          mma_ss_lead(lead, tmem + L::s_col(x), qdesc[x] + off, kd + off, kIdS, kk > 0 ? 1u : 0u);
+          mma_ss_lead(lead, tmem + L::s_col(x), sdesc_join(q_lo + off, kHi), sdesc_join(k_lo + off, kHi), kIdS,
+                      kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv_half = [&](int x, int vst, int h, uint32_t acc0) {   // O_x += P_x[keys of half h] V[same keys]
-        const uint64_t vd = vdesc + uint32_t(vst * (L::TILE >> 4));
+        const uint32_t v_lo = s0 + uint32_t((L::V_OFF + vst * L::TILE) >> 4) + kMN;
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
-          mma_ts_lead(lead, tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, vd + uint32_t(kk * (2048 >> 4)), kIdPV,
-                      kk > 0 ? 1u : acc0);
+          mma_ts_lead(lead, tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_join(v_lo + kk * (2048 >> 4), kHi),
+                      kIdPV, kk > 0 ? 1u : acc0);
       };
       if (!wait(&k_full[gk % KST], (gk / KST) & 1)) { ok = false; break; }
 #pragma unroll

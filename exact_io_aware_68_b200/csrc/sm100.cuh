@@ -262,6 +262,16 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// The same descriptor from its two 32-bit words. High word: stride byte offset, version, layout.
+// Low word: start >> 4 and leading byte offset >> 4 << 16. A buffer at byte offset `off` from a
+// 16-byte-aligned base has low word (base >> 4) + (off >> 4) + sdesc_lbo(lbo): one add when base
+// and off are fixed. The start field must stay below 2^14 (shared addresses below 256 KB).
+__host__ __device__ constexpr uint32_t sdesc_sw128_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__host__ __device__ constexpr uint32_t sdesc_lbo(uint32_t lbo) { return ((lbo >> 4) & 0x3FFFu) << 16; }
+__device__ __forceinline__ uint64_t sdesc_join(uint32_t lo, uint32_t hi) { return (uint64_t(hi) << 32) | lo; }
+
 // TMEM loads/stores, 32 lanes x 32 bits, N consecutive columns per thread.
 #define FA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
                  "=r"(r[i + 6]), "=r"(r[i + 7])
