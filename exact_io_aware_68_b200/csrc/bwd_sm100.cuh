@@ -323,10 +323,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp == 9) {
     // =========================================================== MMA issuer
-    // The whole warp runs the loop (descriptors stay warp-uniform); lane 0 issues every MMA and
-    // commit under a predicate, so one thread owns all tcgen05 work.
+    // The whole warp runs the loop (descriptors stay warp-uniform); the lane that elect.sync picks
+    // issues every MMA and commit, so one thread owns all tcgen05 work.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
-    const uint32_t lead = lane == 0 ? 1u : 0u;
     if (n_iter > 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (V) and Q (dO) K-major
       constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A K-major, B MN-major
@@ -341,20 +340,20 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
-          mma_ss_lead(lead, tmem + L::ST_COL, sdesc_join(k_lo + off, kHi), sdesc_join(q_lo + off, kHi), kIdS,
+          mma_ss_elect(tmem + L::ST_COL, sdesc_join(k_lo + off, kHi), sdesc_join(q_lo + off, kHi), kIdS,
                       kk > 0 ? 1u : 0u);
         }
-        mma_commit_lead(lead, s_full);
+        mma_commit_elect(s_full);
       };
       auto issue_dp = [&](int t) {   // dP^T = V dO_t^T
         const uint32_t v_lo = lo(L::V_OFF, kKM), do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kKM);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
-          mma_ss_lead(lead, tmem + L::DPT_COL, sdesc_join(v_lo + off, kHi), sdesc_join(do_lo + off, kHi), kIdS,
+          mma_ss_elect(tmem + L::DPT_COL, sdesc_join(v_lo + off, kHi), sdesc_join(do_lo + off, kHi), kIdS,
                       kk > 0 ? 1u : 0u);
         }
-        mma_commit_lead(lead, dp_full);
+        mma_commit_elect(dp_full);
       };
       bool ok = warp_wait(kv_full, 0, wc) && warp_wait(&q_full[0], 0, wc);
       if (ok) {
@@ -376,10 +375,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const uint32_t do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kMN);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts_lead(lead, tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_join(do_lo + kk * (2048 >> 4), kHi),
+            mma_ts_elect(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_join(do_lo + kk * (2048 >> 4), kHi),
                         kIdG, kk > 0 ? 1u : acc0);
         }
-        mma_commit_lead(lead, &do_empty[t % DS]);   // dO_t: last read by dV_t
+        mma_commit_elect(&do_empty[t % DS]);   // dO_t: last read by dV_t
         // S_{t+1} over the (P*Z)^T that dV_t has just been given (MMAs run in issue order)
         if (more) {
           if (!warp_wait(&q_full[(t + 1) % QS], ((t + 1) / QS) & 1, wc)) { ok = false; break; }
@@ -393,20 +392,20 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const uint32_t k_lo = lo(L::K_OFF, kMN), ds_lo = lo(L::DS_OFF, kMN);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss_lead(lead, tmem + L::DPT_COL, sdesc_join(k_lo + kk * (2048 >> 4), kHi),
+            mma_ss_elect(tmem + L::DPT_COL, sdesc_join(k_lo + kk * (2048 >> 4), kHi),
                         sdesc_join(ds_lo + kk * (2048 >> 4), kHi), kIdQ, kk > 0 ? 1u : 0u);
         }
-        mma_commit_lead(lead, dq_full);
+        mma_commit_elect(dq_full);
         // dK += dS^T Q_t   (A = dS^T from shared memory, K-major: rows = keys, 16 queries per step)
         {
           const uint32_t ds_lo = lo(L::DS_OFF, kKM), q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kMN);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss_lead(lead, tmem + L::DK_COL, sdesc_join(ds_lo + (((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4), kHi),
+            mma_ss_elect(tmem + L::DK_COL, sdesc_join(ds_lo + (((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4), kHi),
                         sdesc_join(q_lo + kk * (2048 >> 4), kHi), kIdG, kk > 0 ? 1u : acc0);
         }
-        mma_commit_lead(lead, dk_done);             // the dS tile is free again
-        mma_commit_lead(lead, &q_empty[t % QS]);    // Q_t: last read by dK_t
+        mma_commit_elect(dk_done);             // the dS tile is free again
+        mma_commit_elect(&q_empty[t % QS]);    // Q_t: last read by dK_t
         // dP_{t+1} once the dQ warps have read dQ^T out of those columns
         if (more) {
           if (!warp_wait(dq_empty, t & 1, wc)) { ok = false; break; }
@@ -415,8 +414,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           issue_dp(t + 1);
         }
       }
-      mma_commit_lead(lead, fin);
-      if (lead) mbar_drain(fin, 0, p.wait_ns);
+      mma_commit_elect(fin);
+      if (lane == 0) mbar_drain(fin, 0, p.wait_ns);
     }
     __syncwarp();
   } else if (warp < 4) {

@@ -243,10 +243,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp == 9) {
     // =========================================================== MMA issuer
-    // The whole warp runs the loop (descriptors stay warp-uniform); lane 0 issues every MMA and
-    // commit, so one thread owns all tcgen05 work and each commit covers every MMA before it.
+    // The whole warp runs the loop (descriptors stay warp-uniform); the lane that elect.sync picks
+    // issues every MMA and commit, so one thread owns all tcgen05 work and each commit covers
+    // every MMA before it.
     reg_dealloc();
-    const uint32_t lead = lane == 0 ? 1u : 0u;
     auto wait = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc)); };
     constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
     constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
@@ -272,7 +272,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
           const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
-          mma_ss_lead(lead, tmem + L::s_col(x), sdesc_join(q_lo + off, kHi), sdesc_join(k_lo + off, kHi), kIdS,
+          mma_ss_elect(tmem + L::s_col(x), sdesc_join(q_lo + off, kHi), sdesc_join(k_lo + off, kHi), kIdS,
                       kk > 0 ? 1u : 0u);
         }
       };
@@ -280,7 +280,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t v_lo = s0 + uint32_t((L::V_OFF + vst * L::TILE) >> 4) + kMN;
 #pragma unroll
         for (int kk = 4 * h; kk < 4 * h + 4; ++kk)   // 16 keys per step: 8 packed TMEM columns, 2 atoms of V
-          mma_ts_lead(lead, tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_join(v_lo + kk * (2048 >> 4), kHi),
+          mma_ts_elect(tmem + L::o_col(x), tmem + L::s_col(x) + kk * 8, sdesc_join(v_lo + kk * (2048 >> 4), kHi),
                       kIdPV, kk > 0 ? 1u : acc0);
       };
       if (!wait(&k_full[gk % KST], (gk / KST) & 1)) { ok = false; break; }
@@ -291,11 +291,11 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ++nq[x];
         tc_fence_after();
         issue_s(x, gk % KST);
-        mma_commit_lead(lead, &s_full[x]);
-        if (1 == (x ? n_b : n_a)) mma_commit_lead(lead, &q_empty[x]);   // the next item's Q_x may load now
+        mma_commit_elect(&s_full[x]);
+        if (1 == (x ? n_b : n_a)) mma_commit_elect(&q_empty[x]);   // the next item's Q_x may load now
       }
       if (!ok) break;
-      mma_commit_lead(lead, &k_empty[gk % KST]);
+      mma_commit_elect(&k_empty[gk % KST]);
       for (int j = 0; ok && j < n_max; ++j) {
         const int vst = (gv + j) % VST, kst1 = (gk + j + 1) % KST;
         if (!wait(&v_full[vst], ((gv + j) / VST) & 1)) { ok = false; break; }
@@ -320,15 +320,15 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               have_k = true;
             }
             issue_s(x, kst1);
-            mma_commit_lead(lead, &s_full[x]);
-            if (j + 2 == n_x) mma_commit_lead(lead, &q_empty[x]);   // the next item's Q_x may load now
+            mma_commit_elect(&s_full[x]);
+            if (j + 2 == n_x) mma_commit_elect(&q_empty[x]);   // the next item's Q_x may load now
           } else {
-            mma_commit_lead(lead, &o_fin[x]);
+            mma_commit_elect(&o_fin[x]);
           }
         }
         if (!ok) break;
-        mma_commit_lead(lead, &v_empty[vst]);                       // V_j: both tiles' PV issued
-        if (j + 1 < n_max) mma_commit_lead(lead, &k_empty[kst1]);   // K_{j+1}: both tiles' S issued
+        mma_commit_elect(&v_empty[vst]);                       // V_j: both tiles' PV issued
+        if (j + 1 < n_max) mma_commit_elect(&k_empty[kst1]);   // K_{j+1}: both tiles' S issued
       }
       gk += n_max;
       gv += n_max;
@@ -337,8 +337,8 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       ni[0] += (n_a > 0);
       ni[1] += (n_b > 0);
     }
-    mma_commit_lead(lead, fin);   // completes when every MMA issued above has finished
-    if (lead) mbar_drain(fin, 0, p.wait_ns);
+    mma_commit_elect(fin);   // completes when every MMA issued above has finished
+    if (lane == 0) mbar_drain(fin, 0, p.wait_ns);
     __syncwarp();
   } else {
     // =========================================================== softmax / epilogue (warps 0-7)
