@@ -6,5 +6,7 @@ only.  Importing the package does not load the library; the first call does, and
 when it is missing.
 """
 from .api import attention_bwd, attention_fwd, bwd_workspace, check, dropout_mask
+from .autograd import FlashAttentionFunction, flash_attention
 
-__all__ = ["attention_fwd", "attention_bwd", "bwd_workspace", "check", "dropout_mask"]
+__all__ = ["attention_fwd", "attention_bwd", "bwd_workspace", "check", "dropout_mask", "flash_attention",
+           "FlashAttentionFunction"]
