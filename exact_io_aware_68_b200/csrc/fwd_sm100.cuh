@@ -17,8 +17,9 @@
 //              softmax runs, the tensor core works on the other tile.  P is handed over in two
 //              halves of 64 keys, so the first half of PV runs while the second half of P is made.
 // Softmax arithmetic: the scale-and-shift and the row sum use packed f32x2 operations and the row
-// max a tree of three-input maxima; every exponential goes to the MUFU unit (moving a share to a
-// polynomial on the FMA pipe was measured slower: the softmax is bound by instruction issue).
+// max a tree of three-input maxima. At d=128 every exponential goes to the MUFU unit (moving a
+// share to a polynomial on the FMA pipe was measured slower there); at d=64 without dropout a
+// quarter of them take the FMA pipe (see kFmaPairsPer8).
 // TMEM columns: S_A [0,128), S_B [128,256) (P over the first 64 columns of each), O_A [256,256+D),
 // O_B [256+D,256+2D).  tcgen05 operations from one thread complete in issue order, so S_X(j+1)
 // (which overwrites P_X(j)) runs after PV_X(j), and its completion also means PV_X(j) is done.
@@ -84,6 +85,40 @@ __device__ __forceinline__ uint64_t exp2_pair(uint32_t s0, uint32_t s1, uint64_t
   f2_split(x, x0, x1);
   return f2_make(ex2_approx(x0), ex2_approx(x1));
 }
+
+// The same pair on the FMA pipe, so that part of the exponentials leave the MUFU unit (16 results
+// per clock per SM). Range reduction (Cody and Waite): x = n + f with n = floor(x), f in [0, 1);
+// 2^f by a cubic with p(0) = 1 whose coefficients were fitted for this kernel (minimax relative
+// error over [0, 1): 8.6e-5, below the 2^-9 rounding of the bf16 P); 2^n enters by adding n to the
+// exponent field. x is clamped to -127 first: the result is then a subnormal or larger, and the
+// row sum flushes subnormals, so a fully masked row still sums to exactly 0.
+__device__ __forceinline__ uint64_t exp2_pair_fma(uint32_t s0, uint32_t s1, uint64_t sl2x2, uint64_t negm2) {
+  constexpr float kC1 = 0.6951166391372681f, kC2 = 0.22764497995376587f, kC3 = 0.07706724107265472f;
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: adding it leaves floor(x) in the low bits
+  const uint64_t x = f2_fma(f2_make(__uint_as_float(s0), __uint_as_float(s1)), sl2x2, negm2);
+  float x0, x1;
+  f2_split(x, x0, x1);
+  const uint64_t xc = f2_make(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t mg = f2_make(kMagic, kMagic);
+  const uint64_t t = f2_add_rm(xc, mg);                 // kMagic + floor(x), exactly
+  const uint64_t fr = f2_sub(xc, f2_sub(t, mg));        // x - floor(x), exactly
+  uint64_t pp = f2_fma(f2_make(kC3, kC3), fr, f2_make(kC2, kC2));
+  pp = f2_fma(pp, fr, f2_make(kC1, kC1));
+  pp = f2_fma(pp, fr, f2_make(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2_split(pp, p0, p1);
+  f2_split(t, t0, t1);
+  // the low bits of t hold n (two's complement); n << 23 is the exponent increment
+  return f2_make(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+// Of every 8 consecutive score pairs, this many take exp2_pair_fma, the rest the MUFU. Measured on
+// the headline shapes: at d=128 any share was slower (the softmax there is bound by instruction
+// issue and latency); at d=64 without dropout, 2 of 8 made the 64k-token causal forward 8.6 %
+// faster (1 or 3 of 8 less so); with dropout the counter hash already fills the integer and FMA
+// pipes and the share made it slower.
+template <int D, bool DROPOUT>
+constexpr int kFmaPairsPer8 = (D == 64 && !DROPOUT) ? 2 : 0;
 
 __device__ __forceinline__ void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory"); }
 __device__ __forceinline__ void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory"); }
@@ -406,8 +441,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int c = 32 * h + e;   // pair index: keys 2c, 2c+1
-            const uint64_t pp = exp2_pair(sr[2 * c], sr[2 * c + 1], sl2x2, negm2);
-            rs2 = f2_add(rs2, pp);
+            const uint64_t pp = (e % 8) >= 8 - kFmaPairsPer8<D, DROPOUT>
+                                    ? exp2_pair_fma(sr[2 * c], sr[2 * c + 1], sl2x2, negm2)
+                                    : exp2_pair(sr[2 * c], sr[2 * c + 1], sl2x2, negm2);
+            rs2 = kFmaPairsPer8<D, DROPOUT> > 0 ? f2_add_ftz(rs2, pp) : f2_add(rs2, pp);
             float p0, p1;
             f2_split(pp, p0, p1);
             if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
