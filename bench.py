@@ -314,14 +314,21 @@ def run_native(args, w, world, rank, local):
 
 
 def csrc_hash():
-    """Hash of the kernel sources, to tell whether a stored ncu figure still describes them."""
+    """Hash of the kernel code, to tell whether a stored ncu figure still describes it. Comments
+    and whitespace are left out, so editing a comment keeps the figures valid. The sources hold no
+    string literal with comment markers."""
     import glob
     import hashlib
+    import re
 
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_68_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(os.path.basename(f).encode())
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

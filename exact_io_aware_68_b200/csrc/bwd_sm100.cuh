@@ -1,7 +1,7 @@
 // Exact attention backward for sm_100a, recomputing each probability block from Q, K and the
-// saved per-row logsumexp instead of storing P ("48 FlashAttention", block "Backward — тоже без
-// N×N"; "Flash Attention：如何通过硬件感知优化重塑注意力机制的未来", section 2.2: keep only the
-// softmax normalisers and rebuild the attention weights on demand).  Gradients are the exact
+// saved per-row logsumexp instead of storing P ("48 FlashAttention", block "Tiling и online
+// softmax", paragraph "Backward — тоже без N×N"; "Flash Attention：如何通过硬件感知优化重塑注意力机制的
+// 未来", section 2.2: keep only the softmax normalisers and rebuild the attention weights on demand).  Gradients are the exact
 // derivatives of O = dropout(softmax(mask(tau Q K^T))) V:
 //   dV = Pt^T dO,  dPt = dO V^T,  dP = dPt * Z/(1-p),  D_i = rowsum(dO * O)_i,
 //   dS = P * (dP - D),  dQ = tau dS K,  dK = tau dS^T Q.
@@ -10,7 +10,7 @@
 //   fa_bwd_prep_kernel    D = rowsum(dO * O) in fp32, clears the fp32 dQ accumulator
 //   fa_bwd_sm100_kernel   one CTA per (b, h, 128-key tile), K and V resident, loop over query
 //                         tiles; S^T, dP^T, dV, dK, dQ on tcgen05; dQ added into the fp32
-//                         accumulator with vector atomics (fp32 gradient accumulation, as the
+//                         accumulator with TMA bulk reductions (fp32 gradient accumulation, as the
 //                         mixed-precision advice in section 3.2 of the same blog post asks)
 //   fa_bwd_dq_kernel      dQ = bf16(tau * accumulator)
 //
