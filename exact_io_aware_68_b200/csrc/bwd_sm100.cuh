@@ -60,6 +60,7 @@ struct BwdParams {  // (the main kernel also takes tensor maps of q, k, v, dO an
   uint64_t seed;
   uint64_t wait_ns;
   int out_align32;             // dk and dv are 32-byte aligned: epilogues use 32-byte stores
+  int kt_major;                // grid (B*H, n_tiles): key tile = blockIdx.y; else (n_tiles, B*H)
 };
 
 constexpr float kLog2e = 1.4426950408889634074f;
@@ -203,9 +204,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
 
-  // ---- work item: (b, h, key tile kt); heavy causal tiles (small kt) first
-  const int kt = int(blockIdx.x);
-  const int bh = blockIdx.y;
+  // ---- work item: (b, h, key tile kt); the grid order is chosen at launch (kt_major)
+  const int kt = int(p.kt_major ? blockIdx.y : blockIdx.x);
+  const int bh = int(p.kt_major ? blockIdx.x : blockIdx.y);
   const int b = bh / p.H;
   const int k0 = kt * 128;
   int kv_end = p.N;

@@ -178,11 +178,23 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 template <int D, bool DROPOUT>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                          const CUtensorMap& mdq, const fa::BwdParams& p, cudaStream_t s) {
+                          const CUtensorMap& mdq, fa::BwdParams p, cudaStream_t s) {
   using L = fa::BwdLayout<D>;
   fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
-  const dim3 grid(p.n_tiles, p.B * p.H);
+  int sms = 0;
+  if ((st = sm_count(&sms)) != FA_OK) return st;
+  // key-tile-major while the grid has at most 20 CTAs per SM; it then has at most 20 * SMs key
+  // tiles, well inside the 65535 limit of gridDim.y
+  p.kt_major = int64_t(p.B) * p.H * p.n_tiles <= 20 * int64_t(sms) ? 1 : 0;
+  // Blocks are dispatched in linear order. Key-tile-major order (x = head, y = key tile) puts
+  // every head's first key tile (the most query tiles when causal) first, so the one-tile CTAs
+  // form the tail. Head-major order (x = key tile, y = head) keeps the CTAs in flight on a few
+  // heads, so their Q and dO stay in L2, but each head's heaviest CTA starts only when the head
+  // does. That tail is about 2 * SMs / (B*H*n_tiles) of the run: key-tile-major is used while the
+  // grid has at most 20 CTAs per SM (headline causal 2x16x4096x128: 5.7 % faster; 64k-token
+  // sequences, 256 MB of Q and dO: head-major, 9 % faster).
+  const dim3 grid = p.kt_major ? dim3(p.B * p.H, p.n_tiles) : dim3(p.n_tiles, p.B * p.H);
   fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, 384, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status("fa_bwd main kernel launch");
 }
