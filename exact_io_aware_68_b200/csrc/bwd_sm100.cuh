@@ -60,7 +60,8 @@ struct BwdParams {  // (the main kernel also takes tensor maps of q, k, v, dO an
   uint64_t seed;
   uint64_t wait_ns;
   int out_align32;             // dk and dv are 32-byte aligned: epilogues use 32-byte stores
-  int kt_major;                // grid (B*H, n_tiles): key tile = blockIdx.y; else (n_tiles, B*H)
+  int kt_major;                // 1-D grid in head groups, key-tile-major inside a group; else (n_tiles, B*H)
+  int head_group;              // heads per group (kt_major)
 };
 
 constexpr float kLog2e = 1.4426950408889634074f;
@@ -205,8 +206,16 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
 
   // ---- work item: (b, h, key tile kt); the grid order is chosen at launch (kt_major)
-  const int kt = int(p.kt_major ? blockIdx.y : blockIdx.x);
-  const int bh = int(p.kt_major ? blockIdx.x : blockIdx.y);
+  int kt, bh;
+  if (p.kt_major) {   // groups of head_group heads one after another, key-tile-major inside a group
+    const int BH = p.B * p.H, L = int(blockIdx.x), G = p.head_group, per_group = G * p.n_tiles;
+    const int g = L / per_group, r = L % per_group, gs = min(G, BH - g * G);
+    kt = r / gs;
+    bh = g * G + r % gs;
+  } else {
+    kt = int(blockIdx.x);
+    bh = int(blockIdx.y);
+  }
   const int b = bh / p.H;
   const int k0 = kt * 128;
   int kv_end = p.N;
