@@ -21,6 +21,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -87,7 +88,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # the raw samples go to FA_BENCH_CLOCKS_DIR when set (to keep them), else the temp directory
+        log_dir = os.environ.get("FA_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(log_dir, f"fa_bench_clocks_rank{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -109,7 +112,11 @@ class ClockSampler:
             self.proc.kill()
         self.f.close()
         rows = []
-        for line in open(self.path):
+        with open(self.path) as fh:
+            lines = fh.readlines()
+        if not os.environ.get("FA_BENCH_CLOCKS_DIR"):
+            os.remove(self.path)
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 10:
                 continue
