@@ -320,7 +320,7 @@ def run_native(args, w, world, rank, local):
     return line
 
 
-def csrc_hash():
+def csrc_hash(src_dir=None):
     """Hash of the kernel code, to tell whether a stored ncu figure still describes it. Comments
     and whitespace are left out, so editing a comment keeps the figures valid. The sources hold no
     string literal with comment markers."""
@@ -328,8 +328,9 @@ def csrc_hash():
     import hashlib
     import re
 
+    src_dir = src_dir or os.path.join(ROOT, "exact_io_aware_68_b200", "csrc")
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_68_b200", "csrc", "*"))):
+    for f in sorted(glob.glob(os.path.join(src_dir, "*"))):
         with open(f, encoding="utf-8") as fh:
             text = fh.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
