@@ -49,3 +49,14 @@ def test_sampled_rows_are_distinct_and_seeded():
     assert len(set(r.tolist())) == 256 and r.max() < 65536
     np.testing.assert_array_equal(r, sampled_rows(4, 3, 65536, 256))
     assert not np.array_equal(r, sampled_rows(4, 2, 65536, 256))
+
+
+def test_flop_counts_match_the_metric_definition():
+    # 4 N^2 d B H per forward (halved when causal), backward 2.5x: the per-workload figures the
+    # metric is quoted with, in GFLOP (forward, forward + backward)
+    expect = {"bf16_4x16x1024x64": (17.18, 60.13), "bf16_causal_2x16x4096x128": (137.4, 481.0),
+              "bf16_keypad_dropout_16x16x512x64": (17.18, 60.13), "bf16_causal_1x16x65536x64": (8796.0, 30786.0)}
+    for name, (f, fb) in expect.items():
+        w = WORKLOADS[name]
+        assert abs(w.fwd_flops() / 1e9 - f) <= 0.005 * f, name
+        assert abs(w.fwd_bwd_flops() / 1e9 - fb) <= 0.005 * fb, name
