@@ -21,8 +21,8 @@ backward formulas).  Each function names the passage it follows.  Every function
 is pinned by ``tests/test_oracle.py`` against brute force, closed forms, invariants,
 finite differences and published hash vectors; none is "parity unpinned".
 """
-from .attention import allowed_mask, forward, backward, forward_rows, backward_head_blocked
+from .attention import allowed_mask, forward, backward, forward_rows, backward_head_blocked, forward_decode
 from .dropout import keep_mask, keep_threshold
 
-__all__ = ["allowed_mask", "forward", "backward", "forward_rows", "backward_head_blocked",
+__all__ = ["allowed_mask", "forward", "backward", "forward_rows", "backward_head_blocked", "forward_decode",
            "keep_mask", "keep_threshold"]

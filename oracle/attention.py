@@ -168,3 +168,32 @@ def backward_head_blocked(q, k, v, do, scale, causal, key_lens, dropout_p, seed,
         dK += dk
         dV += dv
     return dQ, dK, dV
+
+
+def forward_decode(q, k, v, scale, causal=False, key_lens=None):
+    """O [B,H,Nq,d] and lse [B,H,Nq] for Nq new query rows against a cache of Nkv keys per head.
+
+    The decode use of exact attention ("48 FlashAttention", block "Связи": the kernel under vLLM /
+    PagedAttention; the operation itself is the one of "FlashAttention 的第一原则", section 2).
+    Reading where the page is silent: the cache of sequence b holds L = key_lens[b] valid keys
+    (all Nkv when key_lens is None) and query i of Nq is the token at position L - Nq + i, so
+    causal keeps key j <= L - Nq + i (self-attention's j <= i in absolute positions) and key
+    padding keeps j < L.  A query with no allowed key has O = 0 and lse = -inf.
+    """
+    B, H, Nq, _ = q.shape
+    Nkv = k.shape[2]
+    O = np.zeros((B, H, Nq, v.shape[3]))
+    lse = np.zeros((B, H, Nq))
+    cols = np.arange(Nkv).reshape(1, -1)
+    for b in range(B):
+        L = Nkv if key_lens is None else int(key_lens[b])
+        allowed = np.broadcast_to(cols < L, (Nq, Nkv))
+        if causal:
+            pos = (L - Nq + np.arange(Nq)).reshape(-1, 1)
+            allowed = allowed & (cols <= pos)
+        for h in range(H):
+            S = (q[b, h] @ k[b, h].T) * scale
+            S = np.where(allowed, S, -np.inf)
+            P, _, _, lse[b, h] = _softmax_rows(S)
+            O[b, h] = P @ v[b, h]
+    return O, lse

@@ -336,3 +336,77 @@ def test_tiling_without_rescale_fails_and_online_softmax_matches():
     good = _tiles_online(q[0, 0], k[0, 0], v[0, 0], 1 / 8, 256)
     assert np.abs(bad - O[0, 0]).max() > 1e-1
     np.testing.assert_allclose(good, O[0, 0], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- decode-shaped forward
+def _brute_decode(q, k, v, scale, causal, key_lens):
+    """Scalar loops: query i of Nq is the token at position L - Nq + i of a cache of L valid keys."""
+    B, H, Nq, d = q.shape
+    Nkv, dv = k.shape[2], v.shape[3]
+    O = np.zeros((B, H, Nq, dv))
+    L_ = np.zeros((B, H, Nq))
+    for b in range(B):
+        L = Nkv if key_lens is None else int(key_lens[b])
+        for h in range(H):
+            for i in range(Nq):
+                keys = [j for j in range(Nkv) if j < L and (not causal or j <= L - Nq + i)]
+                if not keys:
+                    L_[b, h, i] = -math.inf
+                    continue
+                s = {j: sum(float(q[b, h, i, c]) * float(k[b, h, j, c]) for c in range(d)) * scale for j in keys}
+                m = max(s.values())
+                e = {j: math.exp(x - m) for j, x in s.items()}
+                tot = sum(e.values())
+                L_[b, h, i] = m + math.log(tot)
+                for j in keys:
+                    for c in range(dv):
+                        O[b, h, i, c] += e[j] / tot * float(v[b, h, j, c])
+    return O, L_
+
+
+@pytest.mark.parametrize("Nq,Nkv,causal,lens", [(1, 7, False, None), (3, 9, True, None), (4, 10, True, [10, 6]),
+                                               (2, 6, False, [4, 0]), (5, 5, True, [5, 3])])
+def test_decode_brute_force(Nq, Nkv, causal, lens):
+    q, k, v = _rand((2, 2, Nq, 4), 60), _rand((2, 2, Nkv, 4), 61), _rand((2, 2, Nkv, 3), 62)
+    kl = None if lens is None else np.array(lens, dtype=np.int32)
+    O, L = oracle.forward_decode(q, k, v, 0.5, causal, kl)
+    Ob, Lb = _brute_decode(q, k, v, 0.5, causal, kl)
+    np.testing.assert_allclose(O, Ob, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(L), np.isneginf(Lb))
+    fin = np.isfinite(Lb)
+    np.testing.assert_allclose(L[fin], Lb[fin], atol=1e-12)
+
+
+def test_decode_rows_equal_the_last_rows_of_causal_self_attention():
+    """The last Nq rows of causal self-attention over N tokens are decode rows against all N keys;
+    with key padding to L, they are rows L - Nq .. L - 1 of causal self-attention over the first L."""
+    N, Nq, d = 40, 6, 8
+    q, k, v = (_rand((1, 2, N, d), s) for s in (63, 64, 65))
+    O, L = oracle.forward(q, k, v, 0.3, True)
+    Od, Ld = oracle.forward_decode(q[:, :, N - Nq:], k, v, 0.3, True)
+    np.testing.assert_allclose(Od, O[:, :, N - Nq:], atol=1e-12)
+    np.testing.assert_allclose(Ld, L[:, :, N - Nq:], atol=1e-12)
+    Lk = 29
+    O2, L2 = oracle.forward(q[:, :, :Lk], k[:, :, :Lk], v[:, :, :Lk], 0.3, True)
+    qd = np.zeros((1, 2, Nq, d))
+    qd[:] = q[:, :, Lk - Nq:Lk]
+    Od2, Ld2 = oracle.forward_decode(qd, k, v, 0.3, True, np.array([Lk], dtype=np.int32))
+    np.testing.assert_allclose(Od2, O2[:, :, Lk - Nq:], atol=1e-12)
+    np.testing.assert_allclose(Ld2, L2[:, :, Lk - Nq:], atol=1e-12)
+
+
+def test_decode_square_non_causal_is_self_attention_and_zero_query_is_a_mean():
+    N, d = 12, 5
+    q, k, v = (_rand((2, 1, N, d), s) for s in (66, 67, 68))
+    O, L = oracle.forward(q, k, v, 0.4)
+    Od, Ld = oracle.forward_decode(q, k, v, 0.4)
+    np.testing.assert_allclose(Od, O, atol=1e-12)
+    np.testing.assert_allclose(Ld, L, atol=1e-12)
+    # q = 0: uniform weights over the allowed keys (causal: j <= L - Nq + i)
+    Nq, Nkv, Lk = 3, 20, 17
+    k2, v2 = _rand((1, 1, Nkv, d), 69), _rand((1, 1, Nkv, d), 70)
+    Oz, Lz = oracle.forward_decode(np.zeros((1, 1, Nq, d)), k2, v2, 0.4, True, np.array([Lk], dtype=np.int32))
+    for i in range(Nq):
+        n_allowed = Lk - Nq + i + 1
+        np.testing.assert_allclose(Oz[0, 0, i], v2[0, 0, :n_allowed].mean(0), atol=1e-12)
+        assert abs(Lz[0, 0, i] - math.log(n_allowed)) < 1e-12
