@@ -81,62 +81,66 @@ def aggregate(step_ms_local, flops_per_step_local, world, reduce_max, reduce_sum
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,utilization.gpu")
+    """SM clock, power and clock-event reasons of one GPU, polled through NVML every ``period_s``
+    from a host thread while the timed region runs (the host has queued the work, so the GPU is busy
+    for the whole window)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        # the raw samples go to FA_BENCH_CLOCKS_DIR when set (to keep them), else the temp directory
-        log_dir = os.environ.get("FA_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(log_dir, f"fa_bench_clocks_rank{gpu_index}_{os.getpid()}.csv")
+    def __init__(self, gpu_index, period_s=0.001):
+        self.gpu, self.period = gpu_index, period_s
+        self.rows, self.thread, self.stop_flag = [], None, False
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
-                                         stderr=subprocess.DEVNULL)
+            import threading
+
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self.thread = None
+            return
+
+        def poll():
+            while not self.stop_flag:
+                try:
+                    self.rows.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                      pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                      pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        rows = []
-        with open(self.path) as fh:
-            lines = fh.readlines()
-        if not os.environ.get("FA_BENCH_CLOCKS_DIR"):
-            os.remove(self.path)
-        for line in lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 10:
-                continue
-            try:
-                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
-                             "active": parts[4], "hw": parts[5], "hwt": parts[6], "swt": parts[7],
-                             "pcap": parts[8], "util": float(parts[9])})
-            except ValueError:
-                continue
+        self.stop_flag = True
+        self.thread.join()
+        rows = [r for r in self.rows if not (r[2] & 0x1)] or self.rows   # drop samples flagged GPU idle
         if not rows:
             return None
-        busy = [r for r in rows if r["util"] > 0] or rows
-        reasons = set()
-        for r in busy:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                              ("pcap", "sw_power_cap")):
-                if r[key].lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": max(r["max"] for r in rows),
-                "reasons": sorted(reasons), "samples": len(busy), "power_w_max": max(r["power"] for r in rows)}
+        reasons = sorted({name for _, _, bits in rows for bit, name in self.REASONS.items() if bits & bit})
+        mhz = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(mhz), "sm_mhz_min": min(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows), "power_w_max": round(max(r[1] for r in rows), 1),
+                "source": "NVML, polled every 1 ms during the timed steps"}
+
+
+# Dense bf16 tensor-core rate of tcgen05 kind::f16 per SM and clock (a 128 x 128 x 16 MMA every
+# 64 cycles; back-to-back MMAs measured 8190 on this part), and NVIDIA's published dense bf16
+# figure for HGX B200.
+TC_FLOP_PER_CLK_SM = 8192
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+def clock_peak_tflops(sm_mhz, sms=148):
+    """Tensor-core peak at the sampled SM clock: 8192 FLOP per clock per SM."""
+    return TC_FLOP_PER_CLK_SM * sms * sm_mhz * 1e6 / 1e12
 
 
 # ----------------------------------------------------------------------------- native arm
@@ -196,12 +200,11 @@ def run_native(args, w, world, rank, local):
     _lib.call("fa_check", sp)
 
     sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.2)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    sampler.start()
     for s in range(args.steps):
         flush.zero_()
         ev[s][0].record(stream)
@@ -278,25 +281,29 @@ def run_native(args, w, world, rank, local):
 
     pk = peaks()
     kflops = {"fa_fwd": w.fwd_flops(), "fa_bwd_main": 2.5 * w.fwd_flops()}
-    # algorithmic HBM bytes of the two HBM-bound launches
-    rows = B * H * N
-    kbytes = {"fa_bwd_prep": rows * d * 2 * 2 + rows * d * 4 + rows * 4,
-              "fa_bwd_dq_convert": rows * d * 4 + rows * d * 2}
+    kbytes = algorithmic_bytes(B, H, N, d)
     kernels = {}
     for n in names:
         entry = {"avg_ms": round(kernel_ms[n], 5), "share": round(kernel_ms[n] / sum(kernel_ms.values()), 4)}
+        gbs = kbytes[n] / (kernel_ms[n] * 1e-3) / 1e9
+        ncu = load_ncu(n, w.name)
         if n in kflops:
             ach = kflops[n] / (kernel_ms[n] * 1e-3) / 1e12
             entry.update({"bound": "tensor", "achieved_tflops": round(ach, 1),
-                          "frac_of_measured_peak": round(ach / pk["bf16_tflops"], 4)})
+                          "frac_of_measured_peak": round(ach / pk["bf16_tflops"], 4),
+                          "hbm_gbs": round(gbs, 1), "hbm_frac_of_measured_peak": round(gbs / pk["hbm_gbs"], 4),
+                          "algorithmic_bytes": kbytes[n],
+                          "tensor_pipe_active_pct": None if ncu is None else ncu.get("tensor_active_pct")})
         else:
-            ach = kbytes[n] / (kernel_ms[n] * 1e-3) / 1e9
-            entry.update({"bound": "hbm", "achieved_gbs": round(ach, 1),
-                          "frac_of_measured_peak": round(ach / pk["hbm_gbs"], 4)})
+            entry.update({"bound": "hbm", "achieved_gbs": round(gbs, 1),
+                          "frac_of_measured_peak": round(gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": kbytes[n]})
+        if ncu is not None:
+            entry["dram_bytes_ncu"] = ncu.get("dram_bytes")
         kernels[n] = entry
     dom = max(kflops, key=lambda n: kernel_ms[n])
     dom_ach = kflops[dom] / (kernel_ms[dom] * 1e-3) / 1e12
-    traffic = load_traffic(dom, w.name)
+    dom_ncu = load_ncu(dom, w.name)
+    mhz = clocks["sm_mhz"] if clocks else None
     line = {
         "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
@@ -305,10 +312,20 @@ def run_native(args, w, world, rank, local):
         "fwd_tflops": round(fwd_tflops, 2), "fwd_ms": round(fwd_ms, 5),
         "fwd_frac_of_peak": round(fwd_tflops / world / pk["bf16_tflops"], 4),
         "fwd_bwd_frac_of_peak": round(tflops / world / pk["bf16_tflops"], 4),
-        "peak_source": f"{pk['source']} bf16 {pk['bf16_tflops']} TFLOP/s (burst), HBM {pk['hbm_gbs']} GB/s",
+        "frac_of_datasheet": {"fwd": round(fwd_tflops / world / DATASHEET_BF16_TFLOPS, 4),
+                              "fwd_bwd": round(tflops / world / DATASHEET_BF16_TFLOPS, 4)},
+        "frac_of_clock_peak": None if mhz is None else {
+            "fwd": round(fwd_tflops / world / clock_peak_tflops(mhz), 4),
+            "fwd_bwd": round(tflops / world / clock_peak_tflops(mhz), 4),
+            "peak_tflops": round(clock_peak_tflops(mhz), 1), "sm_mhz": mhz},
+        "peak_source": (f"targets use the {pk['source']} bf16 peak {pk['bf16_tflops']} TFLOP/s (cuBLAS burst); "
+                        f"HBM {pk['hbm_gbs']} GB/s {pk['source']}; frac_of_datasheet divides by NVIDIA's dense bf16 "
+                        f"{DATASHEET_BF16_TFLOPS} TFLOP/s (HGX B200); frac_of_clock_peak by 8192 FLOP/clk/SM x 148 SMs "
+                        "at the median sampled SM clock"),
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(dom_ach, 1), "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": round(dom_ach / pk["bf16_tflops"], 4), "traffic": traffic,
-                     "algorithmic_flops_per_launch": kflops[dom]},
+                     "unit": "TFLOP/s", "frac": round(dom_ach / pk["bf16_tflops"], 4),
+                     "traffic": None if dom_ncu is None else dom_ncu.get("dram_bytes"),
+                     "algorithmic_flops_per_launch": kflops[dom], "peak_kind": "burst (kernel timed per launch)"},
         "kernels": kernels,
         "e2e": {"value": round(e2e_tflops, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
@@ -340,9 +357,9 @@ def csrc_hash(src_dir=None):
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel, workload):
-    """dram bytes (read + write) per launch of ``kernel`` from the committed ncu summary; None when
-    there is none or the kernel sources changed since it was captured."""
+def load_ncu(kernel, workload):
+    """The committed ncu figures of ``kernel`` on ``workload`` (dram bytes read + written per launch,
+    tensor-pipe active %); None when there are none or the kernel sources changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -351,7 +368,20 @@ def load_traffic(kernel, workload):
     e = d.get(workload, {}).get(kernel)
     if e is None or e.get("csrc_hash") != csrc_hash():
         return None
-    return e["dram_bytes"]
+    return e
+
+
+def algorithmic_bytes(B, H, N, d):
+    """Bytes each launch must move at least (the method's own traffic, no re-reads):
+    fa_fwd reads Q, K, V and writes O (bf16) and lse (fp32); fa_bwd_prep reads O and dO and writes D
+    and clears the fp32 dQ accumulator; fa_bwd_main reads Q, K, V, dO, lse, D and writes dK, dV (its
+    fp32 dQ reductions, 4 B per element and key tile, are the method's choice and not counted);
+    fa_bwd_dq_convert reads the accumulator and writes dQ."""
+    e, rows = B * H * N * d, B * H * N
+    return {"fa_fwd": 4 * 2 * e + 4 * rows,
+            "fa_bwd_prep": 2 * 2 * e + 4 * e + 4 * rows,
+            "fa_bwd_main": 6 * 2 * e + 2 * 4 * rows,
+            "fa_bwd_dq_convert": 4 * e + 2 * e}
 
 
 # ----------------------------------------------------------------------------- oracle timing
@@ -409,6 +439,132 @@ def run_reference(args, w, world, rank):
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------- decode-shaped forward
+def run_decode(args, world, rank, local):
+    """fa_fwd_decode on Nq new rows per head against a cache of Nkv keys (HBM-bound): one step is one
+    call (split + combine launches) over inputs resident in HBM, L2 flushed before each step."""
+    import torch
+    from exact_io_aware_68_b200 import _lib
+    from exact_io_aware_68_b200.inputs import make_decode_inputs
+
+    B, H, Nq, Nkv, d = args.decode
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lib = _lib.load()
+    x = make_decode_inputs(B, H, Nq, Nkv, d, seed=7, exact=False)
+
+    def up(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = up(x["q"]), up(x["k"]), up(x["v"])
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(lib.fa_fwd_decode_workspace_size(B, H, Nq, Nkv, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    a = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Nq, Nkv, d, x["scale"],
+         int(args.decode_causal), None, ws.data_ptr(), ws.numel(), stream.cuda_stream)
+    for _ in range(args.warmup):
+        flush.zero_()
+        _lib.call("fa_fwd_decode", *a)
+    _lib.call("fa_check", stream.cuda_stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        _lib.call("fa_fwd_decode", *a)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    _lib.call("fa_check", stream.cuda_stream)
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    if rank != 0:
+        return None
+    pk = peaks()
+    kv_bytes = 2 * B * H * Nkv * d * 2                      # K and V, bf16, read once
+    alg_bytes = kv_bytes + 2 * B * H * Nq * d * 2 + 4 * B * H * Nq   # + q read, o written, lse written
+    flops = 4.0 * B * H * Nq * Nkv * d                     # upper bound (no causal discount: Nq << Nkv)
+    gbs = alg_bytes / (ms * 1e-3) / 1e9
+    return {"metric": "decode-shaped attention forward, HBM GB/s (K and V read once)", "value": round(gbs, 1),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+            "config": {"workload": f"decode_{B}x{H}_q{Nq}_kv{Nkv}x{d}", "B": B, "H": H, "Nq": Nq, "Nkv": Nkv, "d": d,
+                       "causal": bool(args.decode_causal),
+                       "l2": "flushed (256 MiB write) before each timed step, outside the events"},
+            "roofline": {"kernel": "fa_fwd_decode", "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": None,
+                         "algorithmic_bytes_per_launch": alg_bytes},
+            "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "gpu_launches": 2 * args.steps, "clocks": clocks}
+
+
+# ----------------------------------------------------------------------------- memory against N
+def memory_table(args, local):
+    """Device memory and HBM bytes of exact attention against N, fused (this library) beside a
+    materialising forward + backward made of torch ops (cuBLAS GEMMs, a softmax kernel): the O(N)
+    versus O(N^2) claim of "48 FlashAttention" (block "PyTorch FlashAttention под капотом sdpa") and
+    the memory comparison of "Flash Attention：如何通过硬件感知优化重塑注意力机制的未来" (section 2.1).
+    The materialising arm is a comparison only; it runs where its N x N tensors fit.
+    One JSON line per N: peak bytes allocated during the call beyond the inputs, and the algorithmic
+    HBM bytes (fused: Q, K, V, O, dO, dQ, dK, dV, lse, D; materialising: adds S, P, dP, dS written
+    and read once each, fp32)."""
+    import torch
+    from exact_io_aware_68_b200 import api
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B, H, d = 1, 16, 64
+    for N in (512, 1024, 2048, 4096, 8192, 16384, 32768, 65536):
+        g = torch.Generator(device=dev).manual_seed(N)
+        q, k, v, do = (torch.randn((B, H, N, d), device=dev, generator=g, dtype=torch.float32).to(torch.bfloat16)
+                       for _ in range(4))
+        e = B * H * N * d
+        row = {"N": N, "B": B, "H": H, "d": d}
+        torch.cuda.synchronize(dev)
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        o, lse = api.attention_fwd(q, k, v, None, True)
+        api.attention_bwd(q, k, v, o, lse, do, None, True)
+        t1.record()
+        torch.cuda.synchronize(dev)
+        row["fused_peak_bytes"] = torch.cuda.max_memory_allocated(dev) - base
+        row["fused_hbm_bytes"] = 8 * e + 4 * B * H * N + 16 * e + 8 * B * H * N
+        row["fused_ms"] = round(t0.elapsed_time(t1), 3)
+        del o, lse
+        nn = B * H * N * N
+        row["materialising_hbm_bytes"] = row["fused_hbm_bytes"] + 4 * 2 * 4 * nn   # S, P, dP, dS: fp32, write + read
+        need = 4 * 4 * nn + 8 * e
+        free = torch.cuda.mem_get_info(dev)[0]
+        if need < 0.8 * free:
+            qf, kf, vf = (t.float().requires_grad_() for t in (q, k, v))
+            torch.cuda.synchronize(dev)
+            base = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            t0.record()
+            s_ = (qf @ kf.transpose(-1, -2)) / d ** 0.5
+            s_ = s_.masked_fill(torch.ones(N, N, dtype=torch.bool, device=dev).triu(1), float("-inf"))
+            p_ = torch.softmax(s_, dim=-1)
+            o_ = p_ @ vf
+            o_.backward(do.float())
+            t1.record()
+            torch.cuda.synchronize(dev)
+            row["materialising_peak_bytes"] = torch.cuda.max_memory_allocated(dev) - base
+            row["materialising_ms"] = round(t0.elapsed_time(t1), 3)
+            del qf, kf, vf, s_, p_, o_
+        else:
+            row["materialising_peak_bytes"] = None
+            row["materialising_note"] = f"N x N fp32 tensors need {need / 2**30:.0f} GiB: not run"
+        row["nxn_fp32_bytes_per_tensor"] = 4 * nn
+        print(json.dumps(row), flush=True)
+        del q, k, v, do
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -418,12 +574,23 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", type=int, nargs=5, metavar=("B", "H", "NQ", "NKV", "D"),
+                    help="time the decode-shaped forward instead (Nq rows against a cache of Nkv keys)")
+    ap.add_argument("--decode-causal", type=int, default=1)
+    ap.add_argument("--memory-table", action="store_true",
+                    help="print device memory and HBM bytes against N, fused beside materialising, and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()
+    if args.memory_table:
+        if rank == 0:
+            memory_table(args, local)
+        return
     w = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.decode is not None:
+        line = run_decode(args, world, rank, local) if args.impl == "native" else None
+    elif args.impl == "reference":
         line = run_reference(args, w, world, rank)
     else:
         line = run_native(args, w, world, rank, local)

@@ -25,7 +25,11 @@ SIGNATURES = {
     "fa_bwd_dq_convert": (_I, [_P, _I, _I, _I, _I, _F, _P, _SZ, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P]),
     "fa_bwd_noalloc_max_scratch": (_SZ, []),
+    "fa_fwd_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_fwd_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _SZ, _P]),
+    "fa_bwd_head_group": (_I, [_I, _I, _SZ]),
     "fa_dropout_mask": (_I, [_P, _I, _I, _I, _F, _U64, _P]),
+    "fa_test_exp2_fma": (_I, [_P, _P, _I, _P]),
     "fa_check": (_I, [_P]),
     "fa_get_error": (ctypes.c_char_p, []),
     "fa_set_wait_limit_ns": (None, [_U64]),

@@ -62,6 +62,7 @@ struct BwdParams {  // (the main kernel also takes tensor maps of q, k, v, dO an
   int out_align32;             // dk and dv are 32-byte aligned: epilogues use 32-byte stores
   int kt_major;                // 1-D grid in head groups, key-tile-major inside a group; else (n_tiles, B*H)
   int head_group;              // heads per group (kt_major)
+  int debug_flags;             // bit 1: the producer never delivers the first Q tile (exercises the timeout path)
 };
 
 constexpr float kLog2e = 1.4426950408889634074f;
@@ -113,33 +114,35 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
 }
 
 // ----------------------------------------------------------------------------- main
-template <int D>
+template <int D, bool DROPOUT>
 struct BwdLayout {
   static constexpr int TILE = 128 * D * 2;
   static constexpr int SUB = 128 * 128;
-  static constexpr int QS = 2;                       // Q ring (and per-tile statistics) depth
-  static constexpr int DS = (D == 128) ? 1 : 2;      // dO ring depth: dO_{t+1} is needed only after dV_t
+  static constexpr int QS = 2;                                  // Q ring (and per-tile statistics) depth
+  static constexpr int DS = (D == 128) ? 1 : 2;                  // dO ring depth (dO_{t+1} is needed after dV_t)
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + TILE;
   static constexpr int Q_OFF = V_OFF + TILE;
   static constexpr int DO_OFF = Q_OFF + QS * TILE;
   static constexpr int DS_OFF = DO_OFF + DS * TILE;          // 128 keys x 128 queries bf16, 2 panels
-  static constexpr int STG_OFF = DS_OFF + 2 * SUB;            // dQ staging for the bulk reductions
-  static constexpr int STAT_OFF = STG_OFF + 32768;            // per stage: -lse2[128], -D[128]
+  // dQ staging for the bulk reductions: per dQ warp, QPR queries x FPW features of fp32
+  static constexpr int FPW = (D == 128) ? 32 : 16;            // dQ^T features per warp (TMEM lanes with data)
+  static constexpr int STG_BYTES = (D == 128 && DROPOUT) ? 16384 : 32768;
+  static constexpr int STAGE_BYTES = STG_BYTES / 4;
+  static constexpr int QPR = STAGE_BYTES / (FPW * 4);          // queries per reduction round
+  static constexpr int ROUNDS = 128 / QPR;
+  static constexpr int STG_OFF = DS_OFF + 2 * SUB;
+  static constexpr int KEEP_OFF = STG_OFF + STG_BYTES;       // dropout keep bits: 2 stages x 128 keys x 128 bits
+  static constexpr int STAT_OFF = KEEP_OFF + (DROPOUT ? 2 * 128 * 16 : 0);   // per stage: -lse2[128], -D[128]
   static constexpr int BAR_OFF = STAT_OFF + QS * 1024;
   // kv_full, q_full[QS], q_empty[QS], stat_full[QS], do_full[DS], do_empty[DS], s_full, dp_full,
-  // p_full, ds_full, dq_full, dq_empty, dk_done, fin
-  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 8;
+  // p_full[2], ds_full[2], dq_full, dq_empty, ds_free, fin, keep_full[2]
+  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 10 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
+  // TMEM: S^T, then (P*Z)^T over [0,64); dP^T, then dS^T over [128,192), then dQ^T; dV; dK
   static constexpr int ST_COL = 0, DPT_COL = 128, DV_COL = 256, DK_COL = 256 + D;
   static constexpr int TMEM_COLS = 512;
-  // dQ staging: per warp and round, QPR queries x FPW features of fp32 (8 KB)
-  static constexpr int FPW = (D == 128) ? 32 : 16;     // features per warp (TMEM lanes with data)
-  static constexpr int QPR = (D == 128) ? 64 : 128;    // queries per reduction round
-  static constexpr int ROUNDS = 128 / QPR;
-  static constexpr int STAGE_BYTES = QPR * FPW * 4;
-  static_assert(4 * STAGE_BYTES <= 32768, "dQ staging fits its buffer");
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
@@ -173,12 +176,37 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Keep bits of the 128 query columns of tile `qrow0` for key `key`: bit b of word w is the decision
+// for query qrow0 + 32 w + b.  Counters of consecutive queries are N apart.
+__device__ __forceinline__ uint4 keep_bits_row(const BwdParams& p, uint64_t row_base, int qrow0, int key) {
+  const uint64_t ctr0 = (row_base + uint64_t(qrow0)) * uint64_t(p.N) + uint64_t(key);
+  const uint64_t step = uint64_t(p.N) * kDropGamma;
+  uint64_t z = dropout_z(p.seed, ctr0);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t bits = 0;
+#pragma unroll 8
+    for (int b = 0; b < 32; ++b) {
+      bits |= (dropout_bits_z(z) >= p.drop_thr ? 1u : 0u) << b;
+      z += step;
+    }
+    w[i] = bits;
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Register split per warpgroup (launch: 512 threads x 128 = 65536 registers):
+// 128 x (144 + 144 + 152 + 72) = 65536.
+constexpr int kBwdThreads = 512;
+constexpr int kBwdLaunchRegs = 128;   // the host checks the kernel's register count against this
+
 template <int D, bool DROPOUT>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using L = BwdLayout<D>;
+  using L = BwdLayout<D, DROPOUT>;
   constexpr int QS = L::QS, DS = L::DS;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -195,15 +223,17 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* do_empty = do_full + DS;
   uint64_t* s_full = do_empty + DS;
   uint64_t* dp_full = s_full + 1;
-  uint64_t* p_full = dp_full + 1;
-  uint64_t* ds_full = p_full + 1;
-  uint64_t* dq_full = ds_full + 1;
+  uint64_t* p_full = dp_full + 1;     // [2]: query half
+  uint64_t* ds_full = p_full + 2;     // [2]: query half
+  uint64_t* dq_full = ds_full + 2;
   uint64_t* dq_empty = dq_full + 1;
-  uint64_t* dk_done = dq_empty + 1;
-  uint64_t* fin = dk_done + 1;
+  uint64_t* ds_free = dq_empty + 1;
+  uint64_t* fin = ds_free + 1;
+  uint64_t* keep_full = fin + 1;      // [2]: stage
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
+  uint4* keep_smem = reinterpret_cast<uint4*>(smem + L::KEEP_OFF);   // [2][128]
 
   // ---- work item: (b, h, key tile kt); the grid order is chosen at launch (kt_major)
   int kt, bh;
@@ -236,17 +266,20 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(ds_full, 4);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&p_full[h], 4);
+      mbar_init(&ds_full[h], 4);
+      mbar_init(&keep_full[h], 4);
+    }
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 4);
-    mbar_init(dk_done, 1);
+    mbar_init(ds_free, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -257,13 +290,13 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const WaitCtl wc{p.wait_ns, abort_flag};
   const uint64_t row_base = uint64_t(bh) * uint64_t(p.N);
 
-  // Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
-  // 128 x (248 + 168 + 88) = 64512.  Each role lowers or raises its budget first thing.
-  if (warp == 11) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
-  } else if (warp == 10) {
+  // Register split per warpgroup (launch: 512 threads x 128 = 65536 registers):
+  // 128 x (144 + 144 + 152 + 72) = 65536.  Each role lowers or raises its budget first thing.
+  if (warp == 15) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+  } else if (warp == 14) {
     // =========================================================== per-tile statistics
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
     for (int t = 0; t < n_iter; ++t) {
       const int sq = t % QS;
       const int qrow0 = (q_first + t) * 128;
@@ -285,9 +318,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       mbar_arrive(&stat_full[sq]);
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // =========================================================== producer
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
     if (n_iter > 0) {
       if (lane == 0) {
         prefetch_tmap(&tm_q);
@@ -307,6 +340,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int sq = t % QS, sd = t % DS;
         const int qrow0 = (q_first + t) * 128;
         if (t >= QS && !warp_wait(&q_empty[sq], ((t / QS) - 1) & 1, wc)) break;
+        if (t == 0 && (p.debug_flags & 2)) break;   // test hook: Q tile 0 never arrives
         if (lane == 0) {
           mbar_arrive_expect_tx(&q_full[sq], L::TILE);
 #pragma unroll
@@ -331,14 +365,15 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // =========================================================== MMA issuer
     // The whole warp runs the loop (descriptors stay warp-uniform); the lane that elect.sync picks
-    // issues every MMA and commit, so one thread owns all tcgen05 work.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    // issues every MMA and commit, so one thread owns all tcgen05 work, and the MMAs execute in
+    // issue order: an MMA that overwrites TMEM columns runs after every earlier MMA that reads them.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
     if (n_iter > 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (V) and Q (dO) K-major
-      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A K-major, B MN-major
+      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A in TMEM, B MN-major
       constexpr uint32_t kIdQ = idesc_bf16(D, 128, true, true);       // dQ^T: K^T, dS^T both MN-major
       // descriptors: low word = s0 + (byte offset in shared memory >> 4) + leading-offset field
       // (K-major: 16; MN-major: one 64-column panel)
@@ -378,26 +413,46 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int t = 0; ok && t < n_iter; ++t) {
         const bool more = t + 1 < n_iter;
         const uint32_t acc0 = t > 0 ? 1u : 0u;
-        // dV += (P*Z)^T dO_t   (A = (P*Z)^T in TMEM, B = dO MN-major: N = D, K = queries)
-        if (!warp_wait(p_full, t & 1, wc)) { ok = false; break; }
-        tc_fence_after();
+        // dV += (P*Z)^T dO_t, query half by query half (A = (P*Z)^T in TMEM: half h packed at
+        // columns [64h, 64h+32); B = dO MN-major: N = D, K = 16 queries per step)
         {
           const uint32_t do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kMN);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts_elect(tmem + L::DV_COL, tmem + L::ST_COL + kk * 8, sdesc_join(do_lo + kk * (2048 >> 4), kHi),
-                        kIdG, kk > 0 ? 1u : acc0);
+          for (int h = 0; h < 2; ++h) {
+            if (!warp_wait(&p_full[h], t & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+              mma_ts_elect(tmem + L::DV_COL, tmem + L::ST_COL + 64 * h + (kk & 3) * 8,
+                          sdesc_join(do_lo + kk * (2048 >> 4), kHi), kIdG, kk > 0 ? 1u : acc0);
+          }
+          if (!ok) break;
         }
         mma_commit_elect(&do_empty[t % DS]);   // dO_t: last read by dV_t
-        // S_{t+1} over the (P*Z)^T that dV_t has just been given (MMAs run in issue order)
+        // S_{t+1} over the (P*Z)^T that dV_t has just been given
         if (more) {
           if (!warp_wait(&q_full[(t + 1) % QS], ((t + 1) / QS) & 1, wc)) { ok = false; break; }
           tc_fence_after();
           issue_s(t + 1);
         }
-        // dQ^T = K^T dS^T into the dP^T columns (already read)   (M = D, N = 128 queries, K = 128 keys)
-        if (!warp_wait(ds_full, t & 1, wc)) { ok = false; break; }
-        tc_fence_after();
+        // dK += dS^T Q_t, query half by query half (A = dS^T in TMEM over the dP^T columns, half h
+        // packed at [128 + 64h, 128 + 64h + 32); B = Q MN-major)
+        {
+          const uint32_t q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kMN);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (!warp_wait(&ds_full[h], t & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+              mma_ts_elect(tmem + L::DK_COL, tmem + L::DPT_COL + 64 * h + (kk & 3) * 8,
+                          sdesc_join(q_lo + kk * (2048 >> 4), kHi), kIdG, kk > 0 ? 1u : acc0);
+          }
+          if (!ok) break;
+        }
+        mma_commit_elect(&q_empty[t % QS]);    // Q_t: last read by dK_t
+        // dQ^T = K^T dS^T over the dS^T/dP^T columns, after dK_t has read them
+        // (M = D, N = 128 queries, K = 128 keys; B = dS^T from shared memory)
         {
           const uint32_t k_lo = lo(L::K_OFF, kMN), ds_lo = lo(L::DS_OFF, kMN);
 #pragma unroll
@@ -406,16 +461,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         sdesc_join(ds_lo + kk * (2048 >> 4), kHi), kIdQ, kk > 0 ? 1u : 0u);
         }
         mma_commit_elect(dq_full);
-        // dK += dS^T Q_t   (A = dS^T from shared memory, K-major: rows = keys, 16 queries per step)
-        {
-          const uint32_t ds_lo = lo(L::DS_OFF, kKM), q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kMN);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss_elect(tmem + L::DK_COL, sdesc_join(ds_lo + (((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4), kHi),
-                        sdesc_join(q_lo + kk * (2048 >> 4), kHi), kIdG, kk > 0 ? 1u : acc0);
-        }
-        mma_commit_elect(dk_done);             // the dS tile is free again
-        mma_commit_elect(&q_empty[t % QS]);    // Q_t: last read by dK_t
+        mma_commit_elect(ds_free);             // the shared-memory dS tile is free again
         // dP_{t+1} once the dQ warps have read dQ^T out of those columns
         if (more) {
           if (!warp_wait(dq_empty, t & 1, wc)) { ok = false; break; }
@@ -428,40 +474,48 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (lane == 0) mbar_drain(fin, 0, p.wait_ns);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // =========================================================== compute (key row r)
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 248;\n" ::: "memory");
-    const int r = tid;
+  } else if (warp < 8) {
+    // =========================================================== compute (key row r, query half qh)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 144;\n" ::: "memory");
+    const int qh = warp >> 2;                 // query columns [64 qh, 64 qh + 64) of every tile
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
     const int key = k0 + r;
-    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
-    uint8_t* ds_smem = smem + L::DS_OFF;
+    uint8_t* ds_smem = smem + L::DS_OFF + qh * L::SUB;   // this half's 64 query columns: one panel
     for (int t = 0; t < n_iter; ++t) {
       const int sq = t % QS;
       const int qrow0 = (q_first + t) * 128;
-      const float* st_l = stat + sq * 256;
-      const bool need_mask = (k0 + 128 > kv_end) || (qrow0 + 128 > p.N) || (p.causal && q_first + t == kt);
+      const int qc0 = qrow0 + 64 * qh;         // first query of this half
+      const float* st_l = stat + sq * 256 + 64 * qh;
+      const bool need_mask = (k0 + 128 > kv_end) || (qc0 + 64 > p.N) || (p.causal && q_first + t == kt);
+      uint32_t kb[2] = {0u, 0u};   // dropout keep bits of this key row: query 64 qh + c -> bit c % 32 of kb[c / 32]
+      if (DROPOUT) {
+        if (!warp_wait(&keep_full[t & 1], (t >> 1) & 1, wc)) { ok = false; break; }
+        const uint2 w = reinterpret_cast<const uint2*>(&keep_smem[(t & 1) * 128 + r])[qh];
+        kb[0] = w.x;
+        kb[1] = w.y;
+      }
       if (!warp_wait(s_full, t & 1, wc)) { ok = false; break; }
       if (!warp_wait(&stat_full[sq], (t / QS) & 1, wc)) { ok = false; break; }
       tc_fence_after();
-      // ---- P^T = exp2(S^T tau log2e - lse2): one pass over the 128 query columns
-      float pr[128];
+      // ---- P^T = exp2(S^T tau log2e - lse2) over this half's 64 query columns
+      float pr[64];
       {
         uint32_t* sr = reinterpret_cast<uint32_t*>(pr);
-        tmem_ld32(lane_base + L::ST_COL + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(lane_base + L::ST_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(lane_base + L::ST_COL + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(lane_base + L::ST_COL + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_ld32(lane_base + L::ST_COL + 64 * qh, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(lane_base + L::ST_COL + 64 * qh + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       }
       {
         const uint64_t sl2x2 = f2_make(sl2, sl2);
         const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(st_l);   // pairs of -lse2
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
           float x0, x1;
           f2_split(f2_fma(f2_make(pr[c], pr[c + 1]), sl2x2, nl2[c >> 1]), x0, x1);
           pr[c] = ex2_approx(x0);
@@ -470,62 +524,62 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       if (need_mask) {
         // allowed: key < kv_end, query < N, and (not causal or key <= query)
-        const int lim_q = p.N - qrow0;                                  // query columns < lim_q exist
-        const int from_q = p.causal ? key - qrow0 : -1;                 // causal: columns >= from_q
+        const int lim_q = p.N - qc0;                                    // columns < lim_q exist
+        const int from_q = p.causal ? key - qc0 : -1;                   // causal: columns >= from_q
         const bool key_ok = key < kv_end;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (!key_ok || c >= lim_q || c < from_q) pr[c] = 0.f;
       }
-      uint32_t keep_bits[4] = {0u, 0u, 0u, 0u};
       {
-        const uint64_t drop_col0 = (row_base + uint64_t(qrow0)) * uint64_t(p.N) + uint64_t(key);
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
+        for (int e = 0; e < 32; ++e) {
           float a = pr[2 * e], bb = pr[2 * e + 1];
-          if (DROPOUT) {
-            // element (query i = qrow0 + c, key j = key): ctr = (bh*N + i)*N + j
-            const uint64_t ctr = drop_col0 + uint64_t(2 * e) * uint64_t(p.N);
-            const bool ka = dropout_keep(p.seed, ctr, p.drop_thr);
-            const bool kb = dropout_keep(p.seed, ctr + uint64_t(p.N), p.drop_thr);
-            keep_bits[e >> 4] |= (ka ? 1u : 0u) << (2 * (e & 15));
-            keep_bits[e >> 4] |= (kb ? 1u : 0u) << (2 * (e & 15) + 1);
-            a = ka ? a : 0.f;      // P * Z; dV takes the 1/(1-p) factor in its fp32 epilogue
-            bb = kb ? bb : 0.f;
+          if (DROPOUT) {   // P * Z; dV takes the 1/(1-p) factor in its fp32 epilogue
+            const uint32_t kbits = kb[e >> 4];
+            a = ((kbits >> ((2 * e) & 31)) & 1u) ? a : 0.f;
+            bb = ((kbits >> ((2 * e + 1) & 31)) & 1u) ? bb : 0.f;
           }
           pk[e] = pack_bf16x2(a, bb);
         }
-        // (P*Z)^T overlays the first 64 score columns, already read
-        tmem_st32(lane_base + L::ST_COL + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(lane_base + L::ST_COL + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        // (P*Z)^T over the first 32 of this half's score columns, already read
+        tmem_st32(lane_base + L::ST_COL + 64 * qh, pk);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[qh]);
 
-      // ---- dS^T = P^T * (dP^T Z/(1-p) - D), two halves of 64 query columns
+      // ---- dS^T = P^T * (dP^T Z/(1-p) - D), in chunks of 32 query columns; written twice: as bf16
+      // pairs into TMEM over the dP^T columns already read (the A operand of dK) and into this
+      // half's shared-memory panel (the B operand of dQ^T)
       if (!warp_wait(dp_full, t & 1, wc)) { ok = false; break; }
-      // the dS tile is free: dQ_{t-1} and dK_{t-1} have read it
-      if (t >= 1 && !warp_wait(dk_done, (t - 1) & 1, wc)) { ok = false; break; }
+      // the shared-memory dS tile is free: dQ^T_{t-1} has read it
+      if (t >= 1 && !warp_wait(ds_free, (t - 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
+      if (DROPOUT) {
+        // The keep bits again, through a volatile read: otherwise the compiler keeps the per-column
+        // keep predicates of the P phase alive across the dP wait, which costs registers (spills).
+        const volatile uint32_t* kv =
+            reinterpret_cast<const volatile uint32_t*>(&keep_smem[(t & 1) * 128 + r]) + 2 * qh;
+        kb[0] = kv[0];
+        kb[1] = kv[1];
+      }
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t dr[64];
-        tmem_ld32(lane_base + L::DPT_COL + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-        tmem_ld32(lane_base + L::DPT_COL + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t dr[32];
+        tmem_ld32(lane_base + L::DPT_COL + 64 * qh + 32 * cc, dr);
         tmem_ld_wait();
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-        uint32_t pk[32];
+        reg_fence32(dr);
+        uint32_t pk[16];
         const uint64_t* nd2 = reinterpret_cast<const uint64_t*>(st_l + 128);   // pairs of -D
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = 64 * hh + 2 * e;
+        for (int e = 0; e < 16; ++e) {
+          const int c = 32 * cc + 2 * e;
           float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
           if (DROPOUT) {
-            const uint32_t kbits = keep_bits[c >> 5];
+            const uint32_t kbits = kb[cc];
             dpa = ((kbits >> (c & 31)) & 1u) ? dpa * p.drop_scale : 0.f;
             dpb = ((kbits >> ((c + 1) & 31)) & 1u) ? dpb * p.drop_scale : 0.f;
           }
@@ -533,50 +587,65 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           f2_split(f2_mul(f2_make(pr[c], pr[c + 1]), f2_add(f2_make(dpa, dpb), nd2[c >> 1])), da, db);
           pk[e] = pack_bf16x2(da, db);
         }
-        // dS (queries contiguous) into the 128-byte-swizzled panel hh: row = key r, 16-byte chunks
+        tmem_st16(lane_base + L::DPT_COL + 64 * qh + 16 * cc, pk);
+        // dS (queries contiguous) into the 128-byte-swizzled panel: row = key r, 16-byte chunks of 8
 #pragma unroll
-        for (int chunk = 0; chunk < 8; ++chunk) {   // 8 queries per 16-byte chunk
-          uint4* dst = reinterpret_cast<uint4*>(ds_smem + hh * L::SUB + r * 128 + ((chunk ^ (r & 7)) << 4));
-          *dst = make_uint4(pk[4 * chunk], pk[4 * chunk + 1], pk[4 * chunk + 2], pk[4 * chunk + 3]);
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = 4 * cc + u;
+          uint4* dst = reinterpret_cast<uint4*>(ds_smem + r * 128 + ((chunk ^ (r & 7)) << 4));
+          *dst = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
       fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
-      tc_fence_before();          // (the dP^T loads above precede the dQ MMA that overwrites them)
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) mbar_arrive(&ds_full[qh]);
     }
-    // ---- dV epilogue
+    // ---- dV epilogue: this half of the feature columns
+    constexpr int HD = D / 2;
     if (n_iter == 0) {
       if (key < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dv + (row_base + key) * D);
+        uint4* dst = reinterpret_cast<uint4*>(p.dv + (row_base + key) * D + qh * HD);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < HD / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
       }
     } else if (ok && warp_wait(fin, 0, wc)) {
       tc_fence_after();
       const float s = DROPOUT ? p.drop_scale : 1.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t vr[32];
-        tmem_ld32(lane_base + L::DV_COL + c * 32, vr);
+        tmem_ld32(lane_base + L::DV_COL + qh * HD + c * 32, vr);
         tmem_ld_wait();
         reg_fence32(vr);
-        if (key < p.N) store_row32(p.dv + (row_base + key) * D + c * 32, vr, s, p.out_align32);
+        if (key < p.N) store_row32(p.dv + (row_base + key) * D + qh * HD + c * 32, vr, s, p.out_align32);
       }
     }
   } else {
-    // =========================================================== dQ + dK epilogue (warps 4-7)
+    // =========================================================== dQ + dK epilogue (warps 8-11)
     // TMEM holds dQ^T in the dP^T columns: lane = feature, column = query.  D=128: feature
     // 32*quarter + lane; D=64 (M=64 layout): feature 16*quarter + lane on lanes 0-15.  Each warp
-    // stages its features for QPR queries in its 8 KB slice of the staging buffer ([query][feature],
+    // stages its features for QPR queries in its slice of the staging buffer ([query][feature],
     // fp32) and adds that box to the accumulator with one TMA bulk reduction; the reductions run
-    // in the background while the next tiles are computed.
-    const int quarter = warp - 4;
+    // in the background while the next tiles are computed.  (A red.global.add per element was
+    // measured 25 % slower on the headline backward: the L2 resolves whole-line bulk reductions
+    // faster than word-sized ones.)  With dropout these warps also make the keep bits of the tiles
+    // ahead (two stages in shared memory), so that the compute warps only read them.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 152;\n" ::: "memory");
+    const int quarter = warp - 8;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     float* stage = reinterpret_cast<float*>(smem + L::STG_OFF + quarter * L::STAGE_BYTES);
     const bool lane_ok = lane < L::FPW;
     bool ok = true;
+    if (DROPOUT) {   // keep bits of the first two tiles
+      for (int t = 0; t < 2 && t < n_iter; ++t) {
+        keep_smem[t * 128 + r] = keep_bits_row(p, row_base, (q_first + t) * 128, k0 + r);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&keep_full[t]);
+      }
+    }
     for (int t = 0; t < n_iter; ++t) {
       const int qrow0 = (q_first + t) * 128;
       if (!warp_wait(dq_full, t & 1, wc)) { ok = false; break; }
@@ -602,10 +671,16 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0) {   // rows past N are outside the tensor map and are not written
           tma_reduce_add_3d(&tm_dq, stage, quarter * L::FPW, qrow0 + rd * L::QPR, bh);
           bulk_commit();
         }
+      }
+      // the compute warps have finished tile t (dq_full follows ds_full): its keep-bit stage is free
+      if (DROPOUT && t + 2 < n_iter) {
+        keep_smem[(t & 1) * 128 + r] = keep_bits_row(p, row_base, (q_first + t + 2) * 128, k0 + r);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&keep_full[t & 1]);
       }
     }
     if (lane == 0) bulk_wait0();   // every reduction has completed before the kernel ends
@@ -633,7 +708,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }

@@ -24,4 +24,16 @@ __device__ __forceinline__ bool dropout_keep(uint64_t seed, uint64_t ctr, uint32
   return dropout_bits(seed, ctr) >= thr;
 }
 
+// The same draw from z = seed + (ctr + 1) * gamma already formed, for runs of counters with a fixed
+// stride s: z(ctr + s) = z(ctr) + s * gamma (mod 2^64), one 64-bit add per element.  Only the high
+// word of the last product is needed: (z ^ (z >> 31)) >> 32 = hi ^ (hi >> 31).
+constexpr uint64_t kDropGamma = 0x9E3779B97F4A7C15ull;
+__device__ __forceinline__ uint64_t dropout_z(uint64_t seed, uint64_t ctr) { return seed + (ctr + 1ull) * kDropGamma; }
+__device__ __forceinline__ uint32_t dropout_bits_z(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  const uint32_t hi = uint32_t(z >> 32);
+  return hi ^ (hi >> 31);
+}
+
 }  // namespace fa

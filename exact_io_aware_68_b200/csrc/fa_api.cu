@@ -14,6 +14,7 @@
 
 #include "../../include/fa.h"
 #include "bwd_sm100.cuh"
+#include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "simt_f32.cuh"
 
@@ -54,14 +55,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D view {d, N, B*H} of a bf16 [B,H,N,d] tensor, loaded as 64 x 128 x 1 boxes with the
+// 3-D view {d, N, B*H} of a bf16 [B,H,N,d] tensor, loaded as 64 x box_rows x 1 boxes with the
 // 128-byte swizzle; rows past N (the ragged last tile) read as zeros.
-fa_status make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, const char* name) {
+fa_status make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, const char* name,
+                        unsigned box_rows = 128) {
   auto fn = encode_fn();
   if (fn == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
   const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * cuuint64_t(d) * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -71,13 +73,13 @@ fa_status make_tile_map(CUtensorMap* map, const void* ptr, int BH, int N, int d,
 }
 
 // 3-D view {d, N, B*H} of the fp32 dQ accumulator for the backward's TMA bulk reductions:
-// boxes of (features per warp) x (queries per round), no swizzle; rows past N are not written.
-fa_status make_dq_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+// boxes of (features per dQ warp) x (queries per round), no swizzle; rows past N are not written.
+fa_status make_dq_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, unsigned box_x, unsigned box_y) {
   auto fn = encode_fn();
   if (fn == nullptr) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
   const cuuint64_t strides[2] = {cuuint64_t(d) * 4, cuuint64_t(N) * cuuint64_t(d) * 4};
-  const cuuint32_t box[3] = {d == 128 ? 32u : 16u, d == 128 ? 64u : 128u, 1};
+  const cuuint32_t box[3] = {box_x, box_y, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -92,8 +94,10 @@ fa_status check_common(int B, int H, int N, int d, float scale, float dropout_p,
   if (B < 1 || H < 1 || N < 1) return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1 (got %d, %d, %d)", B, H, N);
   if (int64_t(B) * H > 65535) return fail(FA_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", (long long)B * H);
   if (int64_t(N) > (int64_t(1) << 30)) return fail(FA_ERR_UNSUPPORTED, "N = %d is too large", N);
-  if (d != 64 && d != 128)
-    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: %s supports d in {64, 128}", d, bf16 ? "bf16" : "fp32");
+  if (bf16 && d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: bf16 supports d in {64, 128}", d);
+  if (!bf16 && (d < 1 || d > 128))
+    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: fp32 supports 1 <= d <= 128", d);
   if (!std::isfinite(scale) || !(scale > 0.f)) return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (!(dropout_p >= 0.f) || !(dropout_p < 1.f)) return fail(FA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
   return FA_OK;
@@ -154,10 +158,42 @@ fa_status sm_count(int* out) {
   return FA_OK;
 }
 
+// L2 size of the current device in bytes (queried once per device).
+fa_status l2_bytes(size_t* out) {
+  static std::atomic<long long> cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev >= 0 && dev < 64 && cache[dev].load() > 0) {
+    *out = size_t(cache[dev].load());
+    return FA_OK;
+  }
+  int n = 0;
+  e = cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev);
+  if (e != cudaSuccess || n <= 0) return fail(FA_ERR_CUDA, "cudaDeviceGetAttribute(L2 size): %s", cudaGetErrorString(e));
+  if (dev >= 0 && dev < 64) cache[dev].store(n);
+  *out = size_t(n);
+  return FA_OK;
+}
+
 template <typename K>
 fa_status set_smem(K kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+// The warp-specialised kernels re-split their registers per warpgroup with setmaxnreg; the split
+// adds up to `regs` registers per thread at launch.  A build whose kernel was given fewer
+// registers would leave a setmaxnreg.inc waiting forever, so it is refused before the launch.
+template <typename K>
+fa_status check_launch_regs(K kernel, int regs, const char* name) {
+  cudaFuncAttributes a{};
+  const cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaFuncGetAttributes(%s): %s", name, cudaGetErrorString(e));
+  if (a.numRegs < regs)
+    return fail(FA_ERR_INTERNAL, "%s was built with %d registers per thread; its register split needs %d", name,
+                a.numRegs, regs);
   return FA_OK;
 }
 
@@ -167,21 +203,28 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   using L = fa::FwdLayout<D>;
   fa_status st = set_smem(fa::fa_fwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
+  if ((st = check_launch_regs(fa::fa_fwd_sm100_kernel<D, DROPOUT>, fa::kFwdLaunchRegs, "fa_fwd kernel")) != FA_OK)
+    return st;
   // persistent: one CTA per SM (or fewer when there are fewer work items)
   const long long items = (long long)p.n_pairs * p.B * p.H;
   int sms = 0;
   if ((st = sm_count(&sms)) != FA_OK) return st;
   const dim3 grid(unsigned(items < sms ? items : sms));
-  fa::fa_fwd_sm100_kernel<D, DROPOUT><<<grid, 384, L::BYTES, s>>>(mq, mk, mv, p);
+  fa::fa_fwd_sm100_kernel<D, DROPOUT><<<grid, fa::kFwdThreads, L::BYTES, s>>>(mq, mk, mv, p);
   return launch_status("fa_fwd kernel launch");
 }
 
 template <int D, bool DROPOUT>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                          const CUtensorMap& mdq, fa::BwdParams p, cudaStream_t s) {
-  using L = fa::BwdLayout<D>;
+                          fa::BwdParams p, cudaStream_t s) {
+  using L = fa::BwdLayout<D, DROPOUT>;
+  CUtensorMap mdq;
+  fa_status st0 = make_dq_map(&mdq, p.dq_acc, p.B * p.H, p.N, D, L::FPW, L::QPR);
+  if (st0 != FA_OK) return st0;
   fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D, DROPOUT>, L::BYTES);
   if (st != FA_OK) return st;
+  if ((st = check_launch_regs(fa::fa_bwd_sm100_kernel<D, DROPOUT>, fa::kBwdLaunchRegs, "fa_bwd main kernel")) != FA_OK)
+    return st;
   int sms = 0;
   if ((st = sm_count(&sms)) != FA_OK) return st;
   // Blocks are dispatched in linear order. Head-major order (x = key tile, y = head) keeps the
@@ -193,15 +236,14 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   // A group holds at most 16 heads, and its Q, dO and fp32 dQ accumulator (8*N*d bytes a head)
   // fit in 32 MB of L2. Measured on the headline causal 2x16x4096x128: head-major 352 us,
   // key-tile-major over all 32 heads 332-340 us (2.6x the algorithmic DRAM bytes), groups of 8
-  // heads 330 us. 64k-token sequences keep head-major (the other order was 9 % slower).
+  // heads 330 us. 64k-token sequences keep head-major (the other order was 9 % slower). The group
+  // size comes from the device's L2 size (fa_bwd_head_group).
   p.kt_major = int64_t(p.B) * p.H * p.n_tiles <= 20 * int64_t(sms) ? 1 : 0;
-  {
-    const int64_t per_head = 8 * int64_t(p.N) * D;
-    const int64_t g = (int64_t(32) << 20) / (per_head > 0 ? per_head : 1);
-    p.head_group = int(g < 1 ? 1 : (g > 16 ? 16 : g));
-  }
+  size_t l2 = 0;
+  if ((st = l2_bytes(&l2)) != FA_OK) return st;
+  p.head_group = fa_bwd_head_group(p.N, D, l2);
   const dim3 grid = p.kt_major ? dim3(unsigned(p.B * p.H * p.n_tiles)) : dim3(p.n_tiles, p.B * p.H);
-  fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, 384, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
+  fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, fa::kBwdThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status("fa_bwd main kernel launch");
 }
 
@@ -224,7 +266,43 @@ fa::BwdParams bwd_params(int B, int H, int N, float scale, int causal, const int
   p.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
   p.seed = seed;
   p.wait_ns = g_wait_ns.load();
+  p.debug_flags = g_debug_flags.load();
   return p;
+}
+
+// Key-range split of the decode kernel: about 296 CTAs in all (two per SM of a B200), at least
+// 512 keys per split, in whole 128-key blocks.  Host arithmetic only, so that the workspace size
+// needs no device.
+struct DecodeSplit {
+  int chunk, n_split;
+};
+DecodeSplit decode_split(int BH, int Nkv) {
+  const long long want = (296 + BH - 1) / BH;                        // splits per head
+  long long chunk = (Nkv + want - 1) / want;
+  chunk = (chunk + 127) / 128 * 128;
+  if (chunk < 512) chunk = 512;
+  const long long n = (Nkv + chunk - 1) / chunk;
+  return DecodeSplit{int(chunk), int(n < 1 ? 1 : n)};
+}
+size_t decode_o_bytes(int BH, int n_split, int Nq, int d) {
+  return (size_t(BH) * n_split * Nq * d * 4 + 255) & ~size_t(255);
+}
+size_t decode_ws_bytes(int BH, int Nq, int Nkv, int d) {
+  const DecodeSplit sp = decode_split(BH, Nkv);
+  return decode_o_bytes(BH, sp.n_split, Nq, d) + ((size_t(BH) * sp.n_split * Nq * 2 * 4 + 255) & ~size_t(255));
+}
+
+template <int D>
+fa_status launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecodeParams& p,
+                        cudaStream_t s) {
+  using L = fa::DecodeLayout<D>;
+  fa_status st = set_smem(fa::fa_decode_split_kernel<D>, L::BYTES);
+  if (st != FA_OK) return st;
+  fa::fa_decode_split_kernel<D><<<dim3(p.n_split, p.B * p.H), 192, L::BYTES, s>>>(mq, mk, mv, p);
+  if ((st = launch_status("fa_fwd_decode split kernel launch")) != FA_OK) return st;
+  const unsigned rows = unsigned(p.B * p.H * p.Nq);
+  fa::fa_decode_combine_kernel<D><<<(rows + 7) / 8, 256, 0, s>>>(p);
+  return launch_status("fa_fwd_decode combine kernel launch");
 }
 
 unsigned grid_for(uint64_t work, unsigned per_block) {
@@ -236,8 +314,18 @@ unsigned grid_for(uint64_t work, unsigned per_block) {
 
 extern "C" {
 
+int fa_bwd_head_group(int N, int d, size_t l2_bytes) {
+  // Q, dO (bf16) and the fp32 dQ accumulator of one head: 8 * N * d bytes.  A group fills about a
+  // quarter of L2, rounded to the nearest whole head (measured best on the 126 MB B200: groups of 8
+  // heads at N = 4096, d = 128), 1..16 heads.
+  if (N < 1 || d < 1) return 1;
+  const uint64_t per_head = 8ull * uint64_t(N) * uint64_t(d);
+  const uint64_t g = (uint64_t(l2_bytes) / 4 + per_head / 2) / per_head;
+  return int(g < 1 ? 1 : (g > 16 ? 16 : g));
+}
+
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                 float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream) {
+                 float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream) {
   fa_status st = check_common(B, H, N, d, scale, dropout_p, true);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(q);
@@ -267,13 +355,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.wait_ns = g_wait_ns.load();
   p.debug_flags = g_debug_flags.load();
   p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = stream;
   if (d == 64) return p.dropout ? launch_fwd<64, true>(mq, mk, mv, p, s) : launch_fwd<64, false>(mq, mk, mv, p, s);
   return p.dropout ? launch_fwd<128, true>(mq, mk, mv, p, s) : launch_fwd<128, false>(mq, mk, mv, p, s);
 }
 
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
-                     float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream) {
+                     float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream) {
   fa_status st = check_common(B, H, N, d, scale, dropout_p, false);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(q);
@@ -291,16 +379,21 @@ fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, f
   p.B = B;
   p.H = H;
   p.N = N;
+  p.d = d;
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.dropout = dropout_p > 0.f ? 1 : 0;
   p.drop_thr = drop_threshold(dropout_p);
   p.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
   p.seed = seed;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const dim3 grid((N + 127) / 128, B * H);
-  if (d == 64)
+  cudaStream_t s = stream;
+  const dim3 grid((N + 63) / 64, B * H);   // 64 query rows per CTA
+  if (d <= 32)
+    fa::fa_fwd_f32_kernel<32><<<grid, 128, 0, s>>>(p);
+  else if (d <= 64)
     fa::fa_fwd_f32_kernel<64><<<grid, 128, 0, s>>>(p);
+  else if (d <= 96)
+    fa::fa_fwd_f32_kernel<96><<<grid, 128, 0, s>>>(p);
   else
     fa::fa_fwd_f32_kernel<128><<<grid, 128, 0, s>>>(p);
   return launch_status("fa_fwd_f32 kernel launch");
@@ -312,7 +405,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 }
 
 fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+                      size_t workspace_bytes, cudaStream_t stream) {
   fa_status st = check_common(B, H, N, d, 1.f, 0.f, true);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(o);
@@ -322,7 +415,7 @@ fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d,
   fa::BwdParams p = bwd_params(B, H, N, 1.f, 0, nullptr, 0.f, 0, w);
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.dO = static_cast<const __nv_bfloat16*>(dO);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = stream;
   const uint64_t threads = uint64_t(B) * H * N * (d / 8);
   if (d == 64)
     fa::fa_bwd_prep_kernel<64><<<grid_for(threads, 256), 256, 0, s>>>(p);
@@ -333,7 +426,7 @@ fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d,
 
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
                       int B, int H, int N, int d, float scale, int causal, const int32_t* key_lens, float dropout_p,
-                      uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+                      uint64_t seed, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   fa_status st = check_common(B, H, N, d, scale, dropout_p, true);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(q);
@@ -345,27 +438,26 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* 
   FA_CHECK_PTR(dv);
   Workspace w;
   if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo;
   if ((st = make_tile_map(&mq, q, B * H, N, d, "q")) != FA_OK) return st;
   if ((st = make_tile_map(&mk, k, B * H, N, d, "k")) != FA_OK) return st;
   if ((st = make_tile_map(&mv, v, B * H, N, d, "v")) != FA_OK) return st;
   if ((st = make_tile_map(&mdo, dO, B * H, N, d, "dO")) != FA_OK) return st;
-  if ((st = make_dq_map(&mdq, w.dq_acc, B * H, N, d)) != FA_OK) return st;
   fa::BwdParams p = bwd_params(B, H, N, scale, causal, key_lens, dropout_p, seed, w);
   p.lse = lse;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.out_align32 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = stream;
   if (d == 64)
-    return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, mdq, p, s)
-                     : launch_bwd_main<64, false>(mq, mk, mv, mdo, mdq, p, s);
-  return p.dropout ? launch_bwd_main<128, true>(mq, mk, mv, mdo, mdq, p, s)
-                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, mdq, p, s);
+    return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, s)
+                     : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, s);
+  return p.dropout ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, s)
+                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, s);
 }
 
 fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+                            size_t workspace_bytes, cudaStream_t stream) {
   fa_status st = check_common(B, H, N, d, scale, 0.f, true);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(dq);
@@ -373,9 +465,12 @@ fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, v
   if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
   fa::BwdParams p = bwd_params(B, H, N, scale, 0, nullptr, 0.f, 0, w);
   p.dq = static_cast<__nv_bfloat16*>(dq);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = stream;
   const uint64_t n8 = uint64_t(B) * H * N * d / 8;
-  const unsigned grid = grid_for(n8, 256) > 148u * 16u ? 148u * 16u : grid_for(n8, 256);
+  int sms = 0;
+  if ((st = sm_count(&sms)) != FA_OK) return st;
+  const unsigned cap = unsigned(sms) * 16u;   // grid-stride loop: 16 blocks of 256 threads per SM
+  const unsigned grid = grid_for(n8, 256) > cap ? cap : grid_for(n8, 256);
   if (d == 64)
     fa::fa_bwd_dq_kernel<64><<<grid, 256, 0, s>>>(p);
   else
@@ -385,7 +480,7 @@ fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, v
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
                  void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, const int32_t* key_lens,
-                 float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+                 float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   FA_CHECK_PTR(dq);
   fa_status st = fa_bwd_prep(o, dO, B, H, N, d, workspace, workspace_bytes, stream);
   if (st != FA_OK) return st;
@@ -395,19 +490,74 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   return fa_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
-fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, uint64_t seed, void* stream) {
+size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nkv, int d) {
+  if (B < 1 || H < 1 || Nq < 1 || Nkv < 1 || d < 1) return 0;
+  return decode_ws_bytes(B * H, Nq, Nkv, d);
+}
+
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                        int Nkv, int d, float scale, int causal, const int32_t* key_lens, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  fa_status st = check_common(B, H, Nkv, d, scale, 0.f, true);
+  if (st != FA_OK) return st;
+  if (Nq < 1 || Nq > 64) return fail(FA_ERR_UNSUPPORTED, "Nq = %d: fa_fwd_decode takes 1 <= Nq <= 64", Nq);
+  FA_CHECK_PTR(q);
+  FA_CHECK_PTR(k);
+  FA_CHECK_PTR(v);
+  FA_CHECK_PTR(o);
+  FA_CHECK_PTR(lse);
+  if (workspace == nullptr) return fail(FA_ERR_INVALID_ARG, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FA_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  const size_t need = decode_ws_bytes(B * H, Nq, Nkv, d);
+  if (workspace_bytes < need) return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  const DecodeSplit sp = decode_split(B * H, Nkv);
+  CUtensorMap mq, mk, mv;
+  if ((st = make_tile_map(&mq, q, B * H, Nq, d, "q", 64)) != FA_OK) return st;
+  if ((st = make_tile_map(&mk, k, B * H, Nkv, d, "k")) != FA_OK) return st;
+  if ((st = make_tile_map(&mv, v, B * H, Nkv, d, "v")) != FA_OK) return st;
+  fa::DecodeParams p{};
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_o_bytes(B * H, sp.n_split, Nq, d));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.key_lens = key_lens;
+  p.B = B;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.chunk = sp.chunk;
+  p.n_split = sp.n_split;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = g_wait_ns.load();
+  return d == 64 ? launch_decode<64>(mq, mk, mv, p, stream) : launch_decode<128>(mq, mk, mv, p, stream);
+}
+
+fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, uint64_t seed, cudaStream_t stream) {
   if (keep == nullptr) return fail(FA_ERR_INVALID_ARG, "keep is NULL");
   if (B < 1 || H < 1 || N < 1) return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1");
   if (!(dropout_p >= 0.f) || !(dropout_p < 1.f)) return fail(FA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
   const uint64_t total = uint64_t(B) * H * N * uint64_t(N);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned grid = grid_for(total, 256) > 148u * 32u ? 148u * 32u : grid_for(total, 256);
+  cudaStream_t s = stream;
+  int sms = 0;
+  const fa_status st = sm_count(&sms);
+  if (st != FA_OK) return st;
+  const unsigned cap = unsigned(sms) * 32u;   // grid-stride loop: 32 blocks of 256 threads per SM
+  const unsigned grid = grid_for(total, 256) > cap ? cap : grid_for(total, 256);
   fa::fa_dropout_mask_kernel<<<grid, 256, 0, s>>>(keep, total, seed, drop_threshold(dropout_p));
   return launch_status("fa_dropout_mask kernel launch");
 }
 
-fa_status fa_check(void* stream) {
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+fa_status fa_test_exp2_fma(const float* x, float* y, int n, cudaStream_t stream) {
+  if (x == nullptr || y == nullptr) return fail(FA_ERR_INVALID_ARG, "x or y is NULL");
+  if (n < 1) return fail(FA_ERR_INVALID_ARG, "n must be >= 1");
+  fa::fa_exp2_fma_test_kernel<<<grid_for((uint64_t(n) + 1) / 2, 256), 256, 0, stream>>>(x, y, n);
+  return launch_status("fa_test_exp2_fma kernel launch");
+}
+
+fa_status fa_check(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
   int code = 0;
   e = cudaMemcpyFromSymbol(&code, fa::g_fa_device_status, sizeof(int));
@@ -472,7 +622,7 @@ extern "C" {
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                          void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-                         const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream) {
+                         const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream) {
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need > kNoallocScratchBytes)
     return fail(FA_ERR_INVALID_ARG,

@@ -112,14 +112,28 @@ __device__ __forceinline__ uint64_t exp2_pair_fma(uint32_t s0, uint32_t s1, uint
   return f2_make(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
                  __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
-// Of every 8 consecutive score pairs, this many take exp2_pair_fma, the rest the MUFU. Measured on
-// the headline shapes: at d=128 any share was slower (the softmax there is bound by instruction
-// issue and latency); at d=64 without dropout, 2 of 8 made the 64k-token causal forward 8.6 %
-// faster (1 or 3 of 8 less so); with dropout the counter hash already fills the integer and FMA
-// pipes and the share made it slower.
-template <int D, bool DROPOUT>
-constexpr int kFmaPairsPer8 = (D == 64 && !DROPOUT) ? 2 : 0;
+// Test kernel: y[i] = 2^x[i] by exp2_pair_fma (scale 1, shift 0), for checking its error bound.
+__global__ void __launch_bounds__(256) fa_exp2_fma_test_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (int(blockIdx.x) * 256 + int(threadIdx.x));
+  if (i >= n) return;
+  const float x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float y0, y1;
+  f2_split(exp2_pair_fma(__float_as_uint(x[i]), __float_as_uint(x1), f2_make(1.f, 1.f), f2_make(0.f, 0.f)), y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
 
+// Of every 8 consecutive score pairs, this many take exp2_pair_fma, the rest the MUFU. Measured:
+// at d=64 without dropout, 2 of 8 made the 64k-token causal forward 8.6 % faster (1 or 3 of 8 less
+// so); at d=128 (headline causal 2x16x4096x128) 1, 2 and 3 of 8 gave 126 -> 123, 120 and 122 us;
+// with dropout the counter hash already fills the integer and FMA pipes and a share made it slower.
+template <int D, bool DROPOUT>
+constexpr int kFmaPairsPer8 = DROPOUT ? 0 : 2;
+
+// Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
+// 128 x (200 + 200 + 104) = 64512.  Each role lowers or raises its budget first thing.
+constexpr int kFwdThreads = 384;
+constexpr int kFwdLaunchRegs = 168;   // the host checks the kernel's register count against this
 __device__ __forceinline__ void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory"); }
 __device__ __forceinline__ void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory"); }
 
@@ -132,7 +146,7 @@ __device__ __forceinline__ void fwd_item(int k, int n_pairs, int BH, int& pair, 
 __device__ __forceinline__ int fwd_snake(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
 
 template <int D, bool DROPOUT>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using L = FwdLayout<D>;
@@ -211,8 +225,6 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.wait_ns, abort_flag};
 
-  // Register split per warpgroup (launch: 384 threads x 168 = 64512 registers):
-  // 128 x (200 + 200 + 104) = 64512.  Each role lowers or raises its budget first thing.
   if (warp == 11) {
     // =========================================================== producer of the Q tiles
     reg_dealloc();
@@ -398,6 +410,8 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int n = tile_n_kv(pair, bh, x);
       const int kv_x = tile_kv_end(pair, bh, x);
       const uint64_t drop_row = (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * uint64_t(p.N);
+      // counter-hash state of key 0 of this row; key j adds j * gamma
+      const uint64_t z_row = DROPOUT ? dropout_z(p.seed, drop_row) : 0ull;
       float m_ref = -INFINITY;   // reference max, exp2 domain
       float l = 0.f;
       for (int j = 0; j < n; ++j) {
@@ -435,6 +449,7 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t negm2 = f2_make(-m_use, -m_use);
         uint64_t rs2 = f2_make(0.f, 0.f);
+        const uint64_t z_blk = z_row + uint64_t(k0) * kDropGamma;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {   // two halves of 64 keys; the MMA takes each half as soon as it is ready
           uint32_t pk[32];
@@ -448,9 +463,9 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float p0, p1;
             f2_split(pp, p0, p1);
             if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
-              const uint64_t ctr = drop_row + uint64_t(k0 + 2 * c);
-              p0 = dropout_keep(p.seed, ctr, p.drop_thr) ? p0 : 0.f;
-              p1 = dropout_keep(p.seed, ctr + 1, p.drop_thr) ? p1 : 0.f;
+              const uint64_t z0 = z_blk + uint64_t(2 * c) * kDropGamma;
+              p0 = dropout_bits_z(z0) >= p.drop_thr ? p0 : 0.f;
+              p1 = dropout_bits_z(z0 + kDropGamma) >= p.drop_thr ? p1 : 0.f;
             }
             pk[e] = pack_bf16x2(p0, p1);
           }

@@ -97,3 +97,25 @@ def sampled_rows(seed: int, h: int, N: int, count: int) -> np.ndarray:
     """Query rows checked per head for long contexts: ``default_rng([seed, h]).choice``."""
     rng = np.random.default_rng([seed, h])
     return np.sort(rng.choice(N, size=min(count, N), replace=False))
+
+
+def make_decode_inputs(B: int, H: int, Nq: int, Nkv: int, d: int, seed: int, key_len_range=None,
+                       factor: float = 1.0, exact: bool = True):
+    """Inputs of a decode-shaped call: Nq query rows against a cache of Nkv keys per head.
+
+    One generator ``numpy.random.default_rng(seed)``: q [B,H,Nq,d], then k and v [B,H,Nkv,d],
+    each standard normal x ``factor`` rounded to bf16 like ``make_inputs``; with a key-length range
+    [lo, hi], ``key_lens = rng.integers(lo, hi + 1, B)`` (int32) follows.
+    """
+    rng = np.random.default_rng(seed)
+    out = {"B": B, "H": H, "Nq": Nq, "Nkv": Nkv, "d": d, "scale": 1.0 / float(d) ** 0.5, "seed": seed}
+    for name, n in (("q", Nq), ("k", Nkv), ("v", Nkv)):
+        s, e = draw_tensor(rng, (B, H, n, d), factor, "bf16", exact)
+        out[name] = s
+        out[name + "64"] = e
+    if key_len_range is not None:
+        lo, hi = key_len_range
+        out["key_lens"] = rng.integers(lo, hi + 1, B).astype(np.int32)
+    else:
+        out["key_lens"] = None
+    return out

@@ -26,8 +26,8 @@
  *  - Pointers are DEVICE pointers owned by the caller, 16-byte aligned; the library never
  *    allocates or frees device memory.  Outputs are overwritten, not accumulated.
  *  - scale (tau) must be finite and > 0 (1/sqrt(d) is the usual value).
- *  - bf16 entry points support d in {64, 128}; N >= 1 is arbitrary (tails are zero-filled by
- *    the tile loads and masked); B*H <= 65535.
+ *  - bf16 entry points support d in {64, 128}, fa_fwd_f32 any 1 <= d <= 128; N >= 1 is arbitrary
+ *    (tails are zero-filled by the tile loads and masked); B*H <= 65535.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  The return value reports argument validation and launch errors only.  Errors
  *    found on the device (a bounded wait that ran out) are reported by fa_check().
@@ -45,6 +45,13 @@
 #define FA_API
 #endif
 
+/* The CUDA stream handle, as the CUDA runtime declares it (driver_types.h), so that this header
+ * needs no CUDA include; a driver-API CUstream is the same type.  If the runtime header comes after
+ * this one, the repeated typedef is legal C11 and C++. */
+#ifndef __DRIVER_TYPES_H__
+typedef struct CUstream_st* cudaStream_t;
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -52,29 +59,34 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,  /* a null or misaligned pointer, a size or parameter out of range */
-  FA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement (e.g. d = 96) */
+  FA_ERR_UNSUPPORTED = 2,  /* a valid request this build does not implement (e.g. bf16 with d = 96) */
   FA_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed */
   FA_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out; its outputs are undefined */
   FA_ERR_INTERNAL = 5      /* the device reported an inconsistent launch (e.g. shared memory alignment) */
 } fa_status;
 
-/* Forward, bf16.  Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).
- * q, k, v: bf16 [B,H,N,d].  One kernel launch. */
+/* Forward, bf16 ("48 FlashAttention", block "Tiling и online softmax": tile by tile with a running
+ * row max m and row sum l, O re-expressed when m moves; the operation of "FlashAttention 的第一原则",
+ * section 2).  Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).  q, k, v: bf16 [B,H,N,d].
+ * d in {64, 128}.  One kernel launch. */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int H, int N, int d, float scale, int causal,
-                 const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream);
+                 const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream);
 
-/* Forward, fp32 throughout (CUDA-core FFMA, no TF32), same semantics and layouts with fp32
- * q, k, v, o.  d in {64, 128}.  One kernel launch. */
+/* Forward, fp32 throughout (CUDA-core FFMA, no TF32; the same online softmax), same semantics and
+ * layouts with fp32 q, k, v, o.  Any head dimension 1 <= d <= 128.  One kernel launch. */
 FA_API fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                      int B, int H, int N, int d, float scale, int causal,
-                     const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream);
+                     const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream);
 
 /* Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator [B,H,N,d] followed by
  * D = rowsum(dO * O) fp32 [B,H,N] (each part 256-byte aligned).  0 on invalid sizes. */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
-/* Backward, bf16.  Given q, k, v, the forward's o and lse, and the upstream gradient dO
+/* Backward, bf16 ("48 FlashAttention", block "Tiling и online softmax", paragraph "Backward — тоже
+ * без N×N": every probability block is recomputed from Q, K and the saved normaliser instead of
+ * being stored; "Flash Attention：如何通过硬件感知优化重塑注意力机制的未来", section 3.2: fp32 gradient
+ * accumulation).  Given q, k, v, the forward's o and lse, and the upstream gradient dO
  * (all as produced/consumed by fa_fwd), writes dq, dk, dv (bf16 [B,H,N,d]).
  * workspace: caller-owned device memory of at least fa_bwd_workspace_size() bytes,
  * 256-byte aligned, clobbered; it must not be shared by calls that may overlap.
@@ -83,7 +95,7 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  const void* dO, void* dq, void* dk, void* dv,
                  int B, int H, int N, int d, float scale, int causal,
                  const int32_t* key_lens, float dropout_p, uint64_t seed,
-                 void* workspace, size_t workspace_bytes, void* stream);
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* The three launches of fa_bwd, exposed separately (same arguments, same workspace) so that a
  * caller can time or interleave them.  Calling them in order is equivalent to fa_bwd.
@@ -91,13 +103,13 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
  *  fa_bwd_main:       dK and dV (written), dQ accumulated (fp32) into the workspace.
  *  fa_bwd_dq_convert: dq = bf16(scale * accumulator). */
 FA_API fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d,
-                      void* workspace, size_t workspace_bytes, void* stream);
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
 FA_API fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO,
                       void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                       const int32_t* key_lens, float dropout_p, uint64_t seed,
-                      void* workspace, size_t workspace_bytes, void* stream);
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
 FA_API fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
-                            void* workspace, size_t workspace_bytes, void* stream);
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Backward that allocates nothing, for callers that cannot allocate device memory: a plugin
  * inside another runtime that owns all device memory and hands it no workspace, or a
@@ -114,21 +126,50 @@ FA_API fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float s
 FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                          const void* dO, void* dq, void* dk, void* dv,
                          int B, int H, int N, int d, float scale, int causal,
-                         const int32_t* key_lens, float dropout_p, uint64_t seed, void* stream);
+                         const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream);
 
 /* Size in bytes of fa_bwd_noalloc's static scratch array (48 MiB). */
 FA_API size_t fa_bwd_noalloc_max_scratch(void);
 
+/* Decode-shaped forward, bf16: Nq new query rows per head (1 <= Nq <= 64) against a cache of Nkv
+ * keys ("48 FlashAttention", block "Связи": the attention under vLLM / PagedAttention).
+ * q: bf16 [B,H,Nq,d]; k, v: bf16 [B,H,Nkv,d]; writes o (bf16 [B,H,Nq,d]) and lse (fp32 [B,H,Nq]).
+ * Sequence b holds L = key_lens[b] valid keys (key_lens: int32 [B] on the device, or NULL for all
+ * Nkv); query i is the token at position L - Nq + i, so causal keeps key j <= L - Nq + i and key
+ * padding keeps j < L.  A query with no allowed key gets O = 0 and lse = -inf.  No dropout.
+ * d in {64, 128}.  The key range of each head is split over CTAs that write fp32 partials
+ * (m, l, unnormalised O) into the caller's workspace (at least fa_fwd_decode_workspace_size()
+ * bytes, 256-byte aligned, clobbered; not shared by calls that may overlap), then a second launch
+ * merges them.  Two kernel launches. */
+FA_API size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nkv, int d);
+FA_API fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int Nq, int Nkv, int d, float scale, int causal,
+                        const int32_t* key_lens, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/* Heads per group of the backward's head-grouped launch order for sequence length N and head
+ * dimension d on a device with l2_bytes of L2: a quarter of L2 divided by the bytes of one head's
+ * Q, dO and fp32 dQ accumulator (8 * N * d), rounded to nearest and clamped to [1, 16].  Host-only
+ * arithmetic, exposed so that it can be checked without a GPU. */
+FA_API int fa_bwd_head_group(int N, int d, size_t l2_bytes);
+
 /* Writes the dropout keep decisions (1 = kept, 0 = dropped) of every element into
  * keep (uint8 [B,H,N,N], device).  For testing the counter hash bit for bit. */
 FA_API fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, uint64_t seed,
-                          void* stream);
+                          cudaStream_t stream);
+
+/* Test hook: y[i] = 2^x[i] (fp32 device arrays of n elements) by the polynomial exponential that
+ * the d = 64 forward runs on the FMA pipe for part of its scores (range reduction x = n + f,
+ * a cubic for 2^f with p(0) = 1, n added to the exponent field; x clamped at -127).  Its relative
+ * error is below 8.6e-5 for x >= -126; x <= -127 gives exactly 0; x in (-127, -126) gives a value
+ * below 2^-126.  For checking that bound. */
+FA_API fa_status fa_test_exp2_fma(const float* x, float* y, int n, cudaStream_t stream);
 
 /* Synchronises `stream`, then reads and clears this device's status word.  Returns
  * FA_ERR_TIMEOUT if a bounded wait ran out in any kernel since the last check,
  * FA_ERR_INTERNAL for other device-detected faults, FA_ERR_CUDA if the synchronisation
  * itself failed, FA_OK otherwise. */
-FA_API fa_status fa_check(void* stream);
+FA_API fa_status fa_check(cudaStream_t stream);
 
 /* Description of the last non-OK status returned on the calling thread. */
 FA_API const char* fa_get_error(void);
@@ -137,8 +178,9 @@ FA_API const char* fa_get_error(void);
  * environment variable FA_WAIT_LIMIT_MS overrides the default).  Applies to later launches. */
 FA_API void fa_set_wait_limit_ns(uint64_t ns);
 
-/* Test hook.  Bit 0: the forward's load warp never delivers its first K/V block, so the
- * consumers' bounded waits run out and fa_check() returns FA_ERR_TIMEOUT.  0 = normal. */
+/* Test hook.  Bit 0: the forward's load warp never delivers its first K/V block; bit 1: the
+ * backward's load warp never delivers its first Q tile.  Either way the consumers' bounded waits
+ * run out, the kernel unwinds and fa_check() returns FA_ERR_TIMEOUT.  0 = normal. */
 FA_API void fa_debug_set_flags(int flags);
 
 /* Library version string. */

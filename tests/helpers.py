@@ -49,7 +49,7 @@ def bf16_ulp_half(x):
 
 
 def bf16_product_bound(x, w):
-    """Per-element rounding allowance of a bf16 P.V product for hand-made edge cases.
+    """Per-element rounding allowance of a bf16 P.V product, for the named edge cases that need it.
 
     P enters the tensor core rounded to bf16 (relative error <= 2^-8: 8 significant bits) and O is
     stored as bf16 (<= 2^-8 of |O|), so |O_gpu - O| <= 2^-8 (sum_j Pt_ij |V_j| + |O_i|) plus the
@@ -60,19 +60,39 @@ def bf16_product_bound(x, w):
     return O, 2.0 ** -8 * (np.einsum("bhij,bhjc->bhic", Pt, np.abs(x["v64"])) + np.abs(O))
 
 
-def assert_o_close(o_gpu, o_ref, bar, extra=None):
-    """max |o_gpu - o_ref| <= bar (+ ``extra``, an elementwise allowance for hand-made edge cases,
-    see ``bf16_product_bound``).  An element whose own bf16 output rounding bound exceeds the bar
-    (|o| >= 4 under bf16) is held to that bound plus 1e-3 and reported separately."""
+class OCheck(dict):
+    """Result of ``assert_o_close``: max_err, n_large and the list of large-magnitude misses."""
+
+
+def assert_o_close(o_gpu, o_ref, bar=O_MAX_ABS_BF16, extra=None, large_ok=False):
+    """Every element within ``bar`` (max-abs) of the oracle.
+
+    ``extra``: an elementwise allowance added to the bar; only the named edge cases that measurably
+    need it pass one (see ``bf16_product_bound``).
+
+    ``large_ok``: an element whose own bf16 rounding bound (half an ulp at |o_ref|, 2^-6 for |O| in
+    [4, 8)) exceeds the bar cannot meet it by construction.  With ``large_ok`` such elements are
+    listed separately, each with its oracle value, its GPU value and that bound, and are held to the
+    bound plus 1e-3; without it (the default) they must meet the plain bar like every other element.
+    Returns an OCheck with ``max_err``, ``n_large`` (elements whose bound exceeds the bar),
+    ``large_misses`` (those over the plain bar) and ``max_err_small`` (max error over the others)."""
     err = np.abs(o_gpu - o_ref)
+    large = bf16_ulp_half(o_ref) > bar
+    allowed = np.full(err.shape, float(bar))
     if extra is not None:
-        allowed = bar + extra
-        big = np.zeros_like(err, dtype=bool)
-    else:
-        big = bf16_ulp_half(o_ref) > bar if bar >= 1e-3 else np.zeros_like(err, dtype=bool)
-        allowed = np.where(big, bf16_ulp_half(o_ref) + 1e-3, bar)
+        allowed = allowed + extra
+    if large_ok:
+        allowed = np.where(large, np.maximum(allowed, bf16_ulp_half(o_ref) + 1e-3), allowed)
     bad = err > allowed
-    assert not bad.any(), (f"max err {err.max():.3e} (bar {bar}); {int(bad.sum())} elements over; worst excess "
-                           f"{(err - allowed).max():.3e}; {int(big.sum())} large-magnitude elements held to "
-                           "their bf16 bound")
-    return float(err.max()), int(big.sum())
+    misses = [(tuple(int(i) for i in idx), float(o_ref[idx]), float(o_gpu[idx]), float(bf16_ulp_half(o_ref[idx])))
+              for idx in zip(*np.nonzero(large & (err > bar)))]
+    res = OCheck(max_err=float(err.max()) if err.size else 0.0, n_large=int(large.sum()), large_misses=misses,
+                 max_err_small=float(err[~large].max()) if (~large).any() else 0.0)
+    assert not bad.any(), (f"max err {res['max_err']:.3e} (bar {bar}); {int(bad.sum())} elements over; worst "
+                           f"excess {(err - allowed).max():.3e}; {res['n_large']} elements with |O| >= 4")
+    return res
+
+
+def case_id(w):
+    """Test id of a parity case: shape, causal flag, key padding flag and dropout rate."""
+    return f"{w.B}x{w.H}x{w.N}x{w.d}-c{int(w.causal)}-pad{int(w.key_len_range is not None)}-p{w.dropout_p}"

@@ -8,8 +8,7 @@ import oracle
 from exact_io_aware_68_b200 import api, flash_attention
 from exact_io_aware_68_b200.inputs import make_inputs
 from exact_io_aware_68_b200.workloads import Workload
-from helpers import GRAD_REL_L2, O_MAX_ABS_BF16, assert_o_close, bf16_product_bound, key_lens_device, rel_l2, \
-    to_device, to_f64
+from helpers import GRAD_REL_L2, O_MAX_ABS_BF16, assert_o_close, key_lens_device, rel_l2, to_device, to_f64
 
 
 def wl(B, H, N, d, causal=False, pad=None, p=0.0, seed=11):
@@ -36,8 +35,7 @@ def test_autograd_gradients_match_oracle(w):
     o.backward(do)
     api.check()
     O, _ = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"], w.causal, x["key_lens"], w.dropout_p, x["seed"])
-    _, extra = bf16_product_bound(x, w)
-    assert_o_close(to_f64(o.detach()), O, O_MAX_ABS_BF16, extra=extra)
+    assert_o_close(to_f64(o.detach()), O, O_MAX_ABS_BF16)
     ref = oracle.backward(x["q64"], x["k64"], x["v64"], x["do64"], x["scale"], w.causal, x["key_lens"],
                           w.dropout_p, x["seed"])
     for name, g, r in zip(("dq", "dk", "dv"), (q.grad, k.grad, v.grad), ref):

@@ -39,13 +39,16 @@ def test_full_workload(name):
     dq, dk, dv = api.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, key_lens_device(x), w.dropout_p, w.seed)
     api.check()
     O, L = oracle.forward(x["q64"], x["k64"], x["v64"], w.scale, w.causal, x["key_lens"], w.dropout_p, w.seed)
-    o_err, n_big = assert_o_close(to_f64(o), O, O_MAX_ABS_BF16)
+    # the plain bar on every element; these workloads have no |O| >= 4 element at all
+    res = assert_o_close(to_f64(o), O, O_MAX_ABS_BF16)
+    assert res["n_large"] == 0, res["n_large"]
+    o_err = res["max_err"]
     l_err = float(np.abs(lse.cpu().numpy() - L).max())
     assert l_err <= LSE_MAX_ABS, l_err
     ref = oracle.backward(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, w.causal, x["key_lens"], w.dropout_p,
                           w.seed)
     errs = {n: rel_l2(to_f64(g), r) for n, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref)}
-    print(f"{name}: O max-abs {o_err:.3e} ({n_big} elements |O|>=4), lse {l_err:.3e}, rel-L2 {errs}")
+    print(f"{name}: O max-abs {o_err:.3e}, lse {l_err:.3e}, rel-L2 {errs}")
     for n, e in errs.items():
         assert e <= GRAD_REL_L2, (n, e)
 
@@ -58,19 +61,29 @@ def test_long_context_64k():
     dq, dk, dv = api.attention_bwd(q, k, v, o, lse, do, w.scale, True)
     api.check()
     o64, lse_h = to_f64(o), lse.cpu().numpy()
-    worst, big = 0.0, 0
+    worst, worst_small, big, misses = 0.0, 0.0, 0, []
     t0 = time.time()
     for h in range(w.H):
         rows = sampled_rows(w.seed, h, w.N, w.sample_rows)
         O, L = oracle.forward_rows(x["q64"], x["k64"], x["v64"], w.scale, True, None, 0.0, w.seed, 0, h, rows)
-        e, nb = assert_o_close(o64[0, h, rows], O, O_MAX_ABS_BF16)
-        worst, big = max(worst, e), big + nb
+        # Early causal rows of N(0,1) inputs average few keys, so |O| >= 4 happens; such an element
+        # cannot meet 1e-2 after bf16 rounding (half an ulp is 2^-6).  Those elements are listed
+        # one by one with the oracle value and held to the rounding bound + 1e-3; all others meet 1e-2.
+        res = assert_o_close(o64[0, h, rows], O, O_MAX_ABS_BF16, large_ok=True)
+        worst, worst_small, big = max(worst, res["max_err"]), max(worst_small, res["max_err_small"]), big + res["n_large"]
+        misses += [(h, int(rows[i[0]]), i[1], ref, got, bound) for i, ref, got, bound in res["large_misses"]]
         assert np.abs(lse_h[0, h, rows] - L).max() <= LSE_MAX_ABS
     t1 = time.time()
+    print(f"64k: {big} sampled elements with |O| >= 4; {len(misses)} of them over 1e-2:")
+    for h, row, col, ref, got, bound in misses:
+        print(f"  head {h} row {row} col {col}: oracle {ref:+.6f} gpu {got:+.6f} |err| {abs(got - ref):.3e} "
+              f"bf16 half-ulp {bound:.3e}")
+    assert worst_small <= O_MAX_ABS_BF16
+    assert len(misses) <= 64, len(misses)
     ref = oracle.backward_head_blocked(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, True, None, 0.0, w.seed,
                                        0, 0, block=256)
     errs = {n: rel_l2(to_f64(g)[0, 0], r) for n, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref)}
-    print(f"64k: forward rows max-abs {worst:.3e} ({big} elements |O|>=4) in {t1 - t0:.0f}s; head-0 backward "
+    print(f"64k: forward rows max-abs {worst:.3e} (others {worst_small:.3e}) in {t1 - t0:.0f}s; head-0 backward "
           f"rel-L2 {errs} in {time.time() - t1:.0f}s")
     for n, e in errs.items():
         assert e <= GRAD_REL_L2, (n, e)

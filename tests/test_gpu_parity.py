@@ -13,7 +13,7 @@ from exact_io_aware_68_b200 import _lib, api
 from exact_io_aware_68_b200.inputs import make_inputs
 from exact_io_aware_68_b200.workloads import Workload
 from helpers import (GRAD_REL_L2, LSE_MAX_ABS, O_MAX_ABS_BF16, O_MAX_ABS_F32, assert_o_close, bf16_product_bound,
-                     key_lens_device, rel_l2, run_fwd, to_device, to_f64)
+                     case_id, key_lens_device, rel_l2, run_fwd, to_device, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,15 +30,32 @@ FWD_CASES = [
 ]
 
 
-@pytest.mark.parametrize("w", FWD_CASES, ids=lambda w: f"{w.B}x{w.H}x{w.N}x{w.d}-c{int(w.causal)}-"
-                                                      f"pad{int(w.key_len_range is not None)}-p{w.dropout_p}")
+# Edge cases that measurably need the bf16 product allowance on top of the plain 1e-2 bar (see
+# helpers.bf16_product_bound), each with the reason and the error measured against the plain bar.
+# Every other case meets the plain bar, except single elements with |O| >= 4, whose own bf16
+# rounding bound (2^-6) is above it: those are listed one by one in the output.
+NEEDS_PRODUCT_ALLOWANCE = {
+    # inputs x2: scores x4, so rows concentrate on a few keys and |O| reaches ~8; the bf16 rounding
+    # of P (2^-9 relative) times |V| up to ~9 exceeds 1e-2 (measured max error 2.9e-2 on a B200)
+    "1x3x512x128-c0-pad0-p0.0": "peaked rows with large |V|",
+}
+
+
+@pytest.mark.parametrize("w", FWD_CASES, ids=case_id)
 def test_forward_matches_oracle(w):
     x = make_inputs(w, with_do=False)
     *_, o, lse = run_fwd(x)
     O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"], w.causal, x["key_lens"], w.dropout_p, x["seed"])
-    _, extra = bf16_product_bound(x, w)
-    assert_o_close(to_f64(o), O, O_MAX_ABS_BF16, extra=extra)
-    np.testing.assert_allclose(lse.cpu().numpy(), L, rtol=0, atol=LSE_MAX_ABS)
+    extra = bf16_product_bound(x, w)[1] if case_id(w) in NEEDS_PRODUCT_ALLOWANCE else None
+    res = assert_o_close(to_f64(o), O, O_MAX_ABS_BF16, extra=extra, large_ok=True)
+    l_err = float(np.abs(lse.cpu().numpy() - L).max())
+    print(f"{case_id(w)}: O max-abs {res['max_err']:.3e} (|O| < 4: {res['max_err_small']:.3e}), "
+          f"lse max-abs {l_err:.3e}; {res['n_large']} elements with |O| >= 4, over 1e-2:")
+    for idx, ref, got, bound in res["large_misses"]:
+        print(f"  {idx}: oracle {ref:+.6f} gpu {got:+.6f} |err| {abs(got - ref):.3e} bf16 half-ulp {bound:.3e}")
+    if extra is None:
+        assert res["max_err_small"] <= O_MAX_ABS_BF16
+    assert l_err <= LSE_MAX_ABS, l_err
 
 
 def test_forward_fp32_path():
@@ -55,6 +72,38 @@ def test_forward_fp32_path():
     O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"], True, x["key_lens"], 0.3, 3)
     assert np.abs(o.double().cpu().numpy() - O).max() <= O_MAX_ABS_F32
     np.testing.assert_allclose(lse.cpu().numpy(), L, rtol=0, atol=LSE_MAX_ABS)
+
+
+@pytest.mark.parametrize("d", [1, 20, 32, 96, 100, 128])
+def test_forward_fp32_any_head_dim(d):
+    """fa_fwd_f32 takes any 1 <= d <= 128 (ragged N, masks, dropout), within 1e-5 of the oracle."""
+    w = wl(2, 2, 150, d, causal=(d % 2 == 0), pad=(40, 150), p=0.1 if d > 50 else 0.0, dtype="f32", seed=60 + d)
+    x = make_inputs(w, with_do=False)
+    *_, o, lse = run_fwd(x)
+    O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"], w.causal, x["key_lens"], w.dropout_p, w.seed)
+    err = np.abs(o.double().cpu().numpy() - O).max()
+    assert err <= O_MAX_ABS_F32, err
+    np.testing.assert_allclose(lse.cpu().numpy(), L, rtol=0, atol=LSE_MAX_ABS)
+
+
+def test_fma_pipe_exp2_error_bound():
+    """The polynomial 2^x used for part of the d = 64 scores: relative error < 8.6e-5 (plus fp32
+    rounding) against fp64 for x >= -126, exactly 0 for x <= -127 (masked scores), and below 2^-126
+    in between, over a dense sweep of [-130, 8]."""
+    x = np.concatenate([np.linspace(-130.0, 8.0, 1_000_003), np.arange(-130, 9, dtype=np.float64),
+                        np.array([-127.0, -126.5, -126.0, -1e-7, 0.0, 1e-7, -np.inf])]).astype(np.float32)
+    xd = torch.from_numpy(x).cuda()
+    yd = torch.empty_like(xd)
+    _lib.call("fa_test_exp2_fma", xd.data_ptr(), yd.data_ptr(), x.size, torch.cuda.current_stream().cuda_stream)
+    api.check()
+    y = yd.cpu().numpy().astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    hi = x >= -126.0
+    rel = np.abs(y[hi] - ref[hi]) / ref[hi]
+    assert rel.max() <= 8.6e-5 + 2.0 ** -23, rel.max()
+    assert (y[x <= -127.0] == 0.0).all()
+    mid = (x > -127.0) & (x < -126.0)
+    assert (np.abs(y[mid]) < 2.0 ** -126).all()
 
 
 def test_zero_key_length_rows():
@@ -105,8 +154,7 @@ BWD_CASES = [
 ]
 
 
-@pytest.mark.parametrize("w", BWD_CASES, ids=lambda w: f"{w.B}x{w.H}x{w.N}x{w.d}-c{int(w.causal)}-"
-                                                      f"pad{int(w.key_len_range is not None)}-p{w.dropout_p}")
+@pytest.mark.parametrize("w", BWD_CASES, ids=case_id)
 def test_backward_matches_oracle(w):
     x = make_inputs(w)
     q, k, v, o, lse = run_fwd(x)
@@ -145,6 +193,98 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     *_, o, lse = run_fwd(x)
     O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"])
     assert_o_close(to_f64(o), O, O_MAX_ABS_BF16)
+
+
+def test_backward_bounded_wait_reports_timeout_and_context_survives():
+    """The backward's load warp withholds the first Q tile: every waiting role of the kernel gives up
+    after the 0.1 s limit, the kernel unwinds, fa_check reports the timeout, and the next call is
+    correct."""
+    lib = _lib.load()
+    w = wl(1, 2, 256, 64, causal=True)
+    x = make_inputs(w)
+    q, k, v, o, lse = run_fwd(x)
+    do = to_device(x, "do")
+    lib.fa_set_wait_limit_ns(100_000_000)   # 0.1 s
+    lib.fa_debug_set_flags(2)               # the backward's load warp never delivers Q tile 0
+    try:
+        api.attention_bwd(q, k, v, o, lse, do, w.scale, True)
+        st = lib.fa_check(torch.cuda.current_stream().cuda_stream)
+    finally:
+        lib.fa_debug_set_flags(0)
+        lib.fa_set_wait_limit_ns(0)
+    assert st == _lib.FA_ERR_TIMEOUT
+    dq, dk, dv = api.attention_bwd(q, k, v, o, lse, do, w.scale, True)
+    api.check()
+    ref = oracle.backward(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, True)
+    for g, r in zip((dq, dk, dv), ref):
+        assert rel_l2(to_f64(g), r) <= GRAD_REL_L2
+
+
+GUARD = 4096   # guard bytes on each side of every output and of the workspace
+
+
+def _guarded(nbytes, align, pattern):
+    """A device buffer of ``nbytes`` (start aligned to ``align``) with GUARD bytes of ``pattern`` on
+    both sides.  Returns (the whole uint8 buffer, offset of the payload)."""
+    buf = torch.full((nbytes + 2 * GUARD + align,), pattern, dtype=torch.uint8, device="cuda")
+    off = GUARD + (-(buf.data_ptr() + GUARD)) % align
+    return buf, off
+
+
+@pytest.mark.parametrize("N", [1, 129, 257, 383])
+@pytest.mark.parametrize("d,causal,pad,p", [(64, False, None, 0.0), (128, True, None, 0.0),
+                                            (64, True, (1, 383), 0.2), (128, False, (100, 383), 0.1)])
+def test_outputs_and_workspace_guards_untouched(N, d, causal, pad, p):
+    """Ragged N: o, lse, dq, dk, dv and the backward workspace sit between guard regions of known
+    bytes; the kernels write every payload element and no guard byte (a substitute for a memory
+    checker on the epilogues' and the dQ reductions' edges)."""
+    w = wl(2, 2, N, d, causal=causal, pad=pad, p=p, seed=40 + N)
+    x = make_inputs(w)
+    q, k, v, do = (to_device(x, n) for n in ("q", "k", "v", "do"))
+    kl = key_lens_device(x)
+    B, H = 2, 2
+    n_el = B * H * N * d
+    lib = _lib.load()
+    ws_bytes = lib.fa_bwd_workspace_size(B, H, N, d)
+    bufs = {}
+    for name, nbytes, align in (("o", 2 * n_el, 32), ("lse", 4 * B * H * N, 16), ("dq", 2 * n_el, 32),
+                                ("dk", 2 * n_el, 32), ("dv", 2 * n_el, 32), ("ws", ws_bytes, 256)):
+        bufs[name] = _guarded(nbytes, align, 0xA5) + (nbytes,)
+
+    def view(name, dtype, shape):
+        buf, off, nbytes = bufs[name]
+        return buf[off:off + nbytes].view(dtype).view(shape)
+
+    o = view("o", torch.bfloat16, (B, H, N, d))
+    lse = view("lse", torch.float32, (B, H, N))
+    dq, dk, dv = (view(n, torch.bfloat16, (B, H, N, d)) for n in ("dq", "dk", "dv"))
+    ws = view("ws", torch.uint8, (ws_bytes,))
+    api.attention_fwd(q, k, v, w.scale, causal, kl, p, w.seed, o=o, lse=lse)
+    api.attention_bwd(q, k, v, o, lse, do, w.scale, causal, kl, p, w.seed, workspace=ws, dq=dq, dk=dk, dv=dv)
+    api.check()
+    for name, (buf, off, nbytes) in bufs.items():
+        host = buf.cpu().numpy()
+        assert (host[:off] == 0xA5).all() and (host[off + nbytes:] == 0xA5).all(), f"{name}: guard bytes overwritten"
+    O, L = oracle.forward(x["q64"], x["k64"], x["v64"], w.scale, causal, x["key_lens"], p, w.seed)
+    res = assert_o_close(to_f64(o), O, O_MAX_ABS_BF16, large_ok=True)
+    assert res["max_err_small"] <= O_MAX_ABS_BF16
+    lse_h = lse.cpu().numpy()
+    assert np.array_equal(np.isneginf(lse_h), np.isneginf(L))
+    fin = np.isfinite(L)
+    assert np.abs(lse_h[fin] - L[fin]).max() <= LSE_MAX_ABS
+    ref = oracle.backward(x["q64"], x["k64"], x["v64"], x["do64"], w.scale, causal, x["key_lens"], p, w.seed)
+    for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+        if np.linalg.norm(r) == 0.0:
+            # N = 1: one key per row, P = 1 and dS = P (dP - D) = 0, so dQ = dK = 0 exactly.  The GPU
+            # forms D = rowsum(dO * O) from the stored bf16 O (relative rounding <= 2^-9 per element),
+            # so |dS| <= 2^-8 sum_c |dO_c O_c| and |dQ|, |dK| <= scale |dS| max(|K|, |Q|).
+            o64 = to_f64(o)
+            ds_bound = 2.0 ** -8 * np.abs(x["do64"] * o64).sum(axis=-1)
+            bound = w.scale * ds_bound.max() * max(np.abs(x["k64"]).max(), np.abs(x["q64"]).max())
+            assert np.abs(to_f64(g)).max() <= bound, (name, np.abs(to_f64(g)).max(), bound)
+            continue
+        err = rel_l2(to_f64(g), r)
+        assert err <= GRAD_REL_L2, (name, err)
 
 
 def test_outputs_only_16_byte_aligned():

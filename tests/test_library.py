@@ -67,6 +67,15 @@ def test_host_validation_rejects_before_launch(lib, args, status):
     assert len(lib.fa_get_error()) > 0
 
 
+@pytest.mark.parametrize("d,status", [(0, _lib.FA_ERR_UNSUPPORTED), (129, _lib.FA_ERR_UNSUPPORTED),
+                                      (256, _lib.FA_ERR_UNSUPPORTED)])
+def test_fp32_head_dim_range(lib, d, status):
+    """fa_fwd_f32 takes 1 <= d <= 128; outside that it refuses before touching the (fake) pointers."""
+    fake = 0x2000
+    st = lib.fa_fwd_f32(fake, fake, fake, fake, fake, 1, 1, 16, d, 0.125, 0, None, 0.0, 0, None)
+    assert st == status and b"fp32" in lib.fa_get_error()
+
+
 def test_bwd_workspace_validation(lib):
     fake = 0x2000
     # workspace too small / misaligned are rejected on the host
@@ -84,3 +93,16 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         _lib.load(str(tmp_path / "absent.so"))
+
+
+@pytest.mark.parametrize("l2,N,d,group", [
+    (126 << 20, 4096, 128, 8),     # B200: Q, dO, dQ accumulator of 8 heads (4 MB each) in a quarter of L2
+    (50 << 20, 4096, 128, 3),      # a smaller L2 holds fewer heads
+    (126 << 20, 512, 64, 16),      # short heads: clamped to 16
+    (126 << 20, 65536, 64, 1),     # one 32 MB head fills a quarter of L2 by itself
+    (50 << 20, 1024, 64, 16),
+    (6 << 20, 1024, 64, 3),
+])
+def test_backward_head_group_follows_the_l2_size(lib, l2, N, d, group):
+    assert lib.fa_bwd_head_group(N, d, l2) == group
+    assert lib.fa_bwd_head_group(0, d, l2) == 1
