@@ -7,31 +7,33 @@
 //   dS = P * (dP - D),  dQ = tau dS K,  dK = tau dS^T Q.
 //
 // Three launches:
-//   fa_bwd_prep_kernel    D = rowsum(dO * O) in fp32, clears the fp32 dQ accumulator
-//   fa_bwd_sm100_kernel   one CTA per (b, h, 128-key tile), K and V resident, loop over query
-//                         tiles; S^T, dP^T, dV, dK, dQ on tcgen05; dQ added into the fp32
-//                         accumulator with TMA bulk reductions (fp32 gradient accumulation, as the
-//                         mixed-precision advice in section 3.2 of the same blog post asks)
+//   fa_bwd_prep_kernel    D = rowsum(dO * O) in fp32; clears the fp32 dQ accumulator and the work
+//                         counter of the main launch
+//   fa_bwd_sm100_kernel   persistent, one CTA per SM; work items (b, h, 128-key tile) with K and V
+//                         resident, each looping over its query tiles; S^T, dP^T, dV, dK, dQ on
+//                         tcgen05; dQ added into the fp32 accumulator with TMA bulk reductions (fp32
+//                         gradient accumulation, as the mixed-precision advice in section 3.2 of the
+//                         same blog post asks)
 //   fa_bwd_dq_kernel      dQ = bf16(tau * accumulator)
 //
-// Main kernel roles (12 warps, three warpgroups with their own register budgets):
-//   warps 0-3  compute (248 registers): thread r owns key row r (TMEM lane r).
-//              P^T = exp2(S^T tau log2e - lse2) (packed f32x2 arithmetic), masks, dropout; (P*Z)^T as
-//              bf16 into TMEM over the first 64 score columns (dV takes 1/(1-p) at the end);
-//              dS^T = P^T (dP^T Z/(1-p) - D) as bf16 into shared memory: one swizzled tile that the
-//              dK MMA reads as a K-major A operand and the dQ MMA as an MN-major B operand; dV epilogue
-//   warps 4-7  dQ (168 registers): read the dQ^T tile from TMEM (lane = feature, column = query),
-//              stage it in its own shared-memory buffer and add it to the fp32 accumulator with TMA
-//              bulk reductions, one per warp, running in the background; dK epilogue
-//   warp 8     producer: TMA K, V once; Q (2 deep) and dO (1 deep at D=128, 2 at D=64) per query
-//              tile
-//   warp 9     MMA issuer; warp 10 loads lse and D per query tile; warp 11 idle
-//              (88 registers for warps 8-11)
-// TMEM (512 columns): ST [0,128) S^T, then (P*Z)^T in [0,64); DPT [128,256) dP^T, then dQ^T;
+// Main kernel roles (16 warps, four warpgroups with their own register budgets):
+//   warps 0-7  compute, two warpgroups: thread r of warp w owns key row r (TMEM lane r) for the query
+//              half w / 4 (64 query columns of each tile).  P^T = exp2(S^T tau log2e - lse2), masks,
+//              dropout; (P*Z)^T as bf16 into TMEM over the half's first 32 score columns (dV takes
+//              1/(1-p) at the end); dS^T = P^T (dP^T Z/(1-p) - D) as bf16 into TMEM over the dP^T
+//              columns already read (the A operand of dK) and into a swizzled shared-memory tile (the
+//              B operand of dQ^T); dV epilogue (half of the features each)
+//   warps 8-11 dQ: read the dQ^T tile from TMEM (lane = feature, column = query), stage it in shared
+//              memory and add it to the accumulator with TMA bulk reductions; dK epilogue; with
+//              dropout, the keep bits of the tiles two ahead
+//   warp 12    producer: takes the work items (item queue below), TMA K and V per item, Q (2 deep)
+//              and dO (1 deep at D=128, 2 at D=64) per query tile
+//   warp 13    MMA issuer; warp 14 loads -lse and -D per query tile into shared memory; warp 15 idle
+// TMEM (512 columns): S^T [0,128), then (P*Z)^T; dP^T [128,256), then dS^T, then dQ^T;
 // dV [256,256+D); dK [256+D,256+2D).  MMA order per query tile t:
-//   dV_t, S_{t+1}, dQ_t, dK_t, dP_{t+1}
-// so S_{t+1} is ready when the compute warps finish dS_t, and only dV_t (needs P_t) and dQ_t
-// (needs dS_t) wait on them.
+//   dV_t (per query half), S_{t+1}, dK_t (per query half), dQ^T_t, dP_{t+1}
+// so S_{t+1} runs while the compute warps make dS_t, and dK_t reads dS^T before dQ^T_t overwrites it
+// (MMAs of one thread execute in issue order).
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -63,6 +65,7 @@ struct BwdParams {  // (the main kernel also takes tensor maps of q, k, v, dO an
   int kt_major;                // 1-D grid in head groups, key-tile-major inside a group; else (n_tiles, B*H)
   int head_group;              // heads per group (kt_major)
   int debug_flags;             // bit 1: the producer never delivers the first Q tile (exercises the timeout path)
+  unsigned int* work_ctr;      // items handed out beyond the first one of each CTA (zeroed by the prep kernel)
 };
 
 constexpr float kLog2e = 1.4426950408889634074f;
@@ -71,6 +74,7 @@ constexpr float kLog2e = 1.4426950408889634074f;
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
   constexpr int TPR = D / 8;                       // threads per row, 8 elements (16 bytes) each
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.work_ctr = 0u;   // the main kernel's item counter
   const uint64_t rows = uint64_t(p.B) * p.H * p.N;
   const uint64_t t = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint64_t row = t / TPR;
@@ -134,10 +138,13 @@ struct BwdLayout {
   static constexpr int STG_OFF = DS_OFF + 2 * SUB;
   static constexpr int KEEP_OFF = STG_OFF + STG_BYTES;       // dropout keep bits: 2 stages x 128 keys x 128 bits
   static constexpr int STAT_OFF = KEEP_OFF + (DROPOUT ? 2 * 128 * 16 : 0);   // per stage: -lse2[128], -D[128]
-  static constexpr int BAR_OFF = STAT_OFF + QS * 1024;
+  static constexpr int NQI = 8;                               // item queue depth
+  static constexpr int ITEM_OFF = STAT_OFF + QS * 1024;       // item ids, int32 [NQI]
+  static constexpr int BAR_OFF = ITEM_OFF + NQI * 4;
   // kv_full, q_full[QS], q_empty[QS], stat_full[QS], do_full[DS], do_empty[DS], s_full, dp_full,
-  // p_full[2], ds_full[2], dq_full, dq_empty, ds_free, fin, keep_full[2]
-  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 10 + 2;
+  // p_full[2], ds_full[2], dq_full, dq_empty, ds_free, fin, keep_full[2], kv_empty, dk_free,
+  // item_full[NQI], item_empty[NQI]
+  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 10 + 2 + 2 + 2 * NQI;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   // TMEM: S^T, then (P*Z)^T over [0,64); dP^T, then dS^T over [128,192), then dQ^T; dV; dK
@@ -201,6 +208,88 @@ __device__ __forceinline__ uint4 keep_bits_row(const BwdParams& p, uint64_t row_
 constexpr int kBwdThreads = 512;
 constexpr int kBwdLaunchRegs = 128;   // the host checks the kernel's register count against this
 
+// One work item: the 128-key tile kt of head bh, and the query tiles it meets.
+struct BwdItem {
+  int kt, bh, k0, kv_end, q_first, n_iter;
+  uint64_t row_base;
+};
+
+// Item L of the launch order.  kt_major: groups of head_group heads one after another, key-tile-major
+// inside a group (each head's heaviest causal key tiles start with its group); else head-major.
+__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p, int L) {
+  BwdItem it;
+  if (p.kt_major) {
+    const int BH = p.B * p.H, G = p.head_group, per_group = G * p.n_tiles;
+    const int g = L / per_group, r = L % per_group, gs = min(G, BH - g * G);
+    it.kt = r / gs;
+    it.bh = g * G + r % gs;
+  } else {
+    it.kt = L % p.n_tiles;
+    it.bh = L / p.n_tiles;
+  }
+  it.k0 = it.kt * 128;
+  it.kv_end = p.N;
+  if (p.key_lens != nullptr) it.kv_end = min(it.kv_end, max(p.key_lens[it.bh / p.H], 0));
+  it.q_first = p.causal ? it.kt : 0;
+  it.n_iter = (it.k0 < it.kv_end) ? (p.n_tiles - it.q_first) : 0;
+  it.row_base = uint64_t(it.bh) * uint64_t(p.N);
+  return it;
+}
+
+// The item queue of a CTA: the producer warp takes items from the launch order, its first item
+// statically (item blockIdx.x) and the rest from a global counter as it gets to them, and passes
+// the ids of items that have query tiles to the other roles through a ring in shared memory (-1
+// ends the sequence).  Consumers release a slot as soon as they have read it.
+struct ItemQueue {
+  volatile int* ids;       // [NQI]
+  uint64_t* full;          // [NQI], one arrival (the producer)
+  uint64_t* empty;         // [NQI], one arrival per consumer warp
+  int nq;
+  // the n-th id of the sequence (a bounded wait for the producer to post it); false on abort
+  __device__ __forceinline__ bool peek(int n, int& id, const WaitCtl& wc) const {
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[n % nq], (n / nq) & 1, wc))) return false;
+    id = ids[n % nq];
+    return true;
+  }
+  __device__ __forceinline__ void release(int n, int lane) const {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[n % nq]);
+  }
+};
+
+// Walks the query tiles of the queued items, ahead of the current one: the dQ warps use it to make
+// the dropout keep bits of the tiles two ahead, which may belong to the next item(s).
+struct BwdTileCursor {
+  int n, t;                // queue index and tile of the cursor
+  BwdItem it;
+  bool valid;
+  __device__ __forceinline__ bool load(const BwdParams& p, const ItemQueue& q, const WaitCtl& wc) {
+    int id;
+    if (!q.peek(n, id, wc)) return false;
+    valid = id >= 0;
+    if (valid) it = bwd_item(p, id);
+    return true;
+  }
+  __device__ __forceinline__ bool start(const BwdParams& p, const ItemQueue& q, const WaitCtl& wc) {
+    n = 0;
+    t = 0;
+    return load(p, q, wc);
+  }
+  __device__ __forceinline__ bool advance(const BwdParams& p, const ItemQueue& q, const WaitCtl& wc) {
+    if (!valid) return true;
+    if (++t < it.n_iter) return true;
+    t = 0;
+    ++n;
+    return load(p, q, wc);
+  }
+};
+
+// Persistent: one CTA per SM, each taking items from the item queue above (dynamically balanced:
+// a CTA takes the next item of the launch order when it gets to it).  TMEM is allocated and the
+// barriers are set up once; every barrier phase counts tiles (g) or items (gi) over the whole
+// sequence, so the Q/dO rings, the statistics and the keep bits run on from one item into the next:
+// the next item's first Q and dO tiles load while the previous one finishes, and its K/V load as soon
+// as the previous item's last MMA has read K and V.
 template <int D, bool DROPOUT>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -228,30 +317,18 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* dq_full = ds_full + 2;
   uint64_t* dq_empty = dq_full + 1;
   uint64_t* ds_free = dq_empty + 1;
-  uint64_t* fin = ds_free + 1;
+  uint64_t* fin = ds_free + 1;        // per item: its last MMA has completed
   uint64_t* keep_full = fin + 1;      // [2]: stage
+  uint64_t* kv_empty = keep_full + 2; // per item: K and V may be replaced
+  uint64_t* dk_free = kv_empty + 1;   // per item: the dK epilogue has read the accumulator
+  const ItemQueue queue{reinterpret_cast<volatile int*>(smem + L::ITEM_OFF), dk_free + 1, dk_free + 1 + L::NQI, L::NQI};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
   uint4* keep_smem = reinterpret_cast<uint4*>(smem + L::KEEP_OFF);   // [2][128]
 
-  // ---- work item: (b, h, key tile kt); the grid order is chosen at launch (kt_major)
-  int kt, bh;
-  if (p.kt_major) {   // groups of head_group heads one after another, key-tile-major inside a group
-    const int BH = p.B * p.H, L = int(blockIdx.x), G = p.head_group, per_group = G * p.n_tiles;
-    const int g = L / per_group, r = L % per_group, gs = min(G, BH - g * G);
-    kt = r / gs;
-    bh = g * G + r % gs;
-  } else {
-    kt = int(blockIdx.x);
-    bh = int(blockIdx.y);
-  }
-  const int b = bh / p.H;
-  const int k0 = kt * 128;
-  int kv_end = p.N;
-  if (p.key_lens != nullptr) kv_end = min(kv_end, max(p.key_lens[b], 0));
-  const int q_first = p.causal ? kt : 0;
-  const int n_iter = (k0 < kv_end) ? (p.n_tiles - q_first) : 0;
+  const int G = int(gridDim.x), cta = int(blockIdx.x);
+  const int n_items = p.B * p.H * p.n_tiles;
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
@@ -275,6 +352,12 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(dq_empty, 4);
     mbar_init(ds_free, 1);
     mbar_init(fin, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(dk_free, 4);
+    for (int i = 0; i < L::NQI; ++i) {
+      mbar_init(&queue.full[i], 1);
+      mbar_init(&queue.empty[i], 14);   // stats, MMA, 8 compute and 4 dQ warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -288,81 +371,130 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.wait_ns, abort_flag};
-  const uint64_t row_base = uint64_t(bh) * uint64_t(p.N);
 
-  // Register split per warpgroup (launch: 512 threads x 128 = 65536 registers):
-  // 128 x (144 + 144 + 152 + 72) = 65536.  Each role lowers or raises its budget first thing.
   if (warp == 15) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
   } else if (warp == 14) {
     // =========================================================== per-tile statistics
     asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
-    for (int t = 0; t < n_iter; ++t) {
-      const int sq = t % QS;
-      const int qrow0 = (q_first + t) * 128;
-      // the stage is reused once dK of tile t-QS (after every read of its statistics) is done
-      if (t >= QS && !warp_wait(&q_empty[sq], ((t / QS) - 1) & 1, wc)) break;
-      // negated: -lse in the exp2 domain and -D
-      float* st_l = stat + sq * 256;
+    int g = 0;   // query tiles so far (all items)
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      int id;
+      if (!queue.peek(n, id, wc)) break;
+      queue.release(n, lane);
+      if (id < 0) break;
+      const BwdItem it = bwd_item(p, id);
+      for (int t = 0; t < it.n_iter; ++t, ++g) {
+        const int sq = g % QS;
+        const int qrow0 = (it.q_first + t) * 128;
+        // the stage is reused once dK of tile g-QS (after every read of its statistics) is done
+        if (g >= QS && !warp_wait(&q_empty[sq], ((g / QS) - 1) & 1, wc)) { ok = false; break; }
+        // negated: -lse in the exp2 domain and -D; one 16-byte store per lane and array
+        float* st_l = stat + sq * 256;
+        float lv[4], dv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c = lane * 4 + e;
-        const int q = qrow0 + c;
-        float lv = 0.f, dv = 0.f;
-        if (q < p.N) {
-          lv = -p.lse[row_base + q] * kLog2e;
-          dv = -p.dvec[row_base + q];
+        for (int e = 0; e < 4; ++e) {
+          const int q = qrow0 + lane * 4 + e;
+          lv[e] = q < p.N ? -p.lse[it.row_base + q] * kLog2e : 0.f;
+          dv[e] = q < p.N ? -p.dvec[it.row_base + q] : 0.f;
         }
-        st_l[c] = lv;
-        st_l[128 + c] = dv;
+        reinterpret_cast<float4*>(st_l)[lane] = make_float4(lv[0], lv[1], lv[2], lv[3]);
+        reinterpret_cast<float4*>(st_l + 128)[lane] = make_float4(dv[0], dv[1], dv[2], dv[3]);
+        mbar_arrive(&stat_full[sq]);
       }
-      mbar_arrive(&stat_full[sq]);
     }
   } else if (warp == 12) {
     // =========================================================== producer
     asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
-    if (n_iter > 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      prefetch_tmap(&tm_dq);
+    }
+    int g = 0, gi = 0;           // query tiles and items with tiles so far
+    int issued_q = 0, issued_do = 0;
+    bool ok = true;
+    auto load_q_do = [&](const BwdItem& it, int t) -> bool {   // tile t of item it, global tile g
+      const int sq = g % QS, sd = g % DS;
+      const int qrow0 = (it.q_first + t) * 128;
+      if (g >= QS && !warp_wait(&q_empty[sq], ((g / QS) - 1) & 1, wc)) return false;
+      if (g == 0 && (p.debug_flags & 2)) return false;   // test hook: the first Q tile never arrives
       if (lane == 0) {
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
-        prefetch_tmap(&tm_do);
-        prefetch_tmap(&tm_dq);
+        mbar_arrive_expect_tx(&q_full[sq], L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + L::Q_OFF + sq * L::TILE + c * L::SUB, &tm_q, &q_full[sq], c * 64, qrow0, it.bh);
+      }
+      issued_q = g + 1;
+      if (g >= DS && !warp_wait(&do_empty[sd], ((g / DS) - 1) & 1, wc)) return false;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&do_full[sd], L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + L::DO_OFF + sd * L::TILE + c * L::SUB, &tm_do, &do_full[sd], c * 64, qrow0, it.bh);
+      }
+      issued_do = g + 1;
+      ++g;
+      return true;
+    };
+    int n_posted = 0;   // ids posted to the item queue
+    auto post = [&](int id) -> bool {
+      if (n_posted >= L::NQI && !warp_wait(&queue.empty[n_posted % L::NQI], ((n_posted / L::NQI) - 1) & 1, wc))
+        return false;
+      if (lane == 0) {
+        queue.ids[n_posted % L::NQI] = id;
+        mbar_arrive(&queue.full[n_posted % L::NQI]);
+      }
+      __syncwarp();
+      ++n_posted;
+      return true;
+    };
+    for (int taken = 0; ok; ++taken) {
+      int id = cta;
+      if (taken > 0) {
+        unsigned int c = 0;
+        if (lane == 0) c = atomicAdd(p.work_ctr, 1u);
+        id = G + int(__shfl_sync(0xffffffffu, c, 0));
+      }
+      if (id >= n_items) break;
+      const BwdItem it = bwd_item(p, id);
+      if (it.n_iter == 0) {
+        // a key tile past the key length: no gradient flows into it, its dK and dV rows are zero
+        for (int e = lane; e < 128 * (D / 8); e += 32) {
+          const int row = it.k0 + e / (D / 8), c = e % (D / 8);
+          if (row < p.N) {
+            reinterpret_cast<uint4*>(p.dk + (it.row_base + row) * D)[c] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(p.dv + (it.row_base + row) * D)[c] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        continue;
+      }
+      if (!post(id)) { ok = false; break; }
+      // the item's first Q and dO tiles need only ring slots: load them before waiting for K/V
+      if (!load_q_do(it, 0)) { ok = false; break; }
+      // K and V replace the previous item's once its last MMA has read them
+      if (gi >= 1 && !warp_wait(kv_empty, (gi - 1) & 1, wc)) { ok = false; break; }
+      if (lane == 0) {
         mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + L::K_OFF + c * L::SUB, &tm_k, kv_full, c * 64, k0, bh);
-          tma_load_3d(smem + L::V_OFF + c * L::SUB, &tm_v, kv_full, c * 64, k0, bh);
+          tma_load_3d(smem + L::K_OFF + c * L::SUB, &tm_k, kv_full, c * 64, it.k0, it.bh);
+          tma_load_3d(smem + L::V_OFF + c * L::SUB, &tm_v, kv_full, c * 64, it.k0, it.bh);
         }
       }
-      int issued_q = 0, issued_do = 0;
-      for (int t = 0; t < n_iter; ++t) {
-        const int sq = t % QS, sd = t % DS;
-        const int qrow0 = (q_first + t) * 128;
-        if (t >= QS && !warp_wait(&q_empty[sq], ((t / QS) - 1) & 1, wc)) break;
-        if (t == 0 && (p.debug_flags & 2)) break;   // test hook: Q tile 0 never arrives
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full[sq], L::TILE);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + L::Q_OFF + sq * L::TILE + c * L::SUB, &tm_q, &q_full[sq], c * 64, qrow0, bh);
-        }
-        issued_q = t + 1;
-        if (t >= DS && !warp_wait(&do_empty[sd], ((t / DS) - 1) & 1, wc)) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&do_full[sd], L::TILE);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem + L::DO_OFF + sd * L::TILE + c * L::SUB, &tm_do, &do_full[sd], c * 64, qrow0, bh);
-        }
-        issued_do = t + 1;
-      }
-      if (lane == 0) {
-        mbar_drain(kv_full, 0, p.wait_ns);
-        for (int t = max(0, issued_q - QS); t < issued_q; ++t) mbar_drain(&q_full[t % QS], (t / QS) & 1, p.wait_ns);
-        for (int t = max(0, issued_do - DS); t < issued_do; ++t)
-          mbar_drain(&do_full[t % DS], (t / DS) & 1, p.wait_ns);
-      }
+      ++gi;
+      for (int t = 1; t < it.n_iter; ++t)
+        if (!load_q_do(it, t)) { ok = false; break; }
+    }
+    if (ok) post(-1);   // end of the sequence
+    // every copy started here lands before the CTA releases its shared memory
+    if (lane == 0) {
+      if (gi >= 1) mbar_drain(kv_full, (gi - 1) & 1, p.wait_ns);
+      for (int t = max(0, issued_q - QS); t < issued_q; ++t) mbar_drain(&q_full[t % QS], (t / QS) & 1, p.wait_ns);
+      for (int t = max(0, issued_do - DS); t < issued_do; ++t) mbar_drain(&do_full[t % DS], (t / DS) & 1, p.wait_ns);
     }
     __syncwarp();
   } else if (warp == 13) {
@@ -371,55 +503,63 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // issues every MMA and commit, so one thread owns all tcgen05 work, and the MMAs execute in
     // issue order: an MMA that overwrites TMEM columns runs after every earlier MMA that reads them.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
-    if (n_iter > 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (V) and Q (dO) K-major
-      constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A in TMEM, B MN-major
-      constexpr uint32_t kIdQ = idesc_bf16(D, 128, true, true);       // dQ^T: K^T, dS^T both MN-major
-      // descriptors: low word = s0 + (byte offset in shared memory >> 4) + leading-offset field
-      // (K-major: 16; MN-major: one 64-column panel)
-      const uint32_t s0 = smem_u32(smem) >> 4;
-      constexpr uint32_t kHi = sdesc_sw128_hi(1024), kKM = sdesc_lbo(16), kMN = sdesc_lbo(L::SUB);
-      auto lo = [&](int off, uint32_t lbo) { return s0 + uint32_t(off >> 4) + lbo; };
-      auto issue_s = [&](int t) {   // S^T = K Q_t^T  (M = 128 keys, N = 128 queries, K = D)
-        const uint32_t k_lo = lo(L::K_OFF, kKM), q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kKM);
+    constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // K (V) and Q (dO) K-major
+    constexpr uint32_t kIdG = idesc_bf16(128, D, false, true);      // dV, dK: A in TMEM, B MN-major
+    constexpr uint32_t kIdQ = idesc_bf16(D, 128, true, true);       // dQ^T: K^T, dS^T both MN-major
+    // descriptors: low word = s0 + (byte offset in shared memory >> 4) + leading-offset field
+    // (K-major: 16; MN-major: one 64-column panel)
+    const uint32_t s0 = smem_u32(smem) >> 4;
+    constexpr uint32_t kHi = sdesc_sw128_hi(1024), kKM = sdesc_lbo(16), kMN = sdesc_lbo(L::SUB);
+    auto lo = [&](int off, uint32_t lbo) { return s0 + uint32_t(off >> 4) + lbo; };
+    auto issue_s = [&](int g) {   // S^T = K Q_g^T  (M = 128 keys, N = 128 queries, K = D)
+      const uint32_t k_lo = lo(L::K_OFF, kKM), q_lo = lo(L::Q_OFF + (g % QS) * L::TILE, kKM);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
-          mma_ss_elect(tmem + L::ST_COL, sdesc_join(k_lo + off, kHi), sdesc_join(q_lo + off, kHi), kIdS,
-                      kk > 0 ? 1u : 0u);
-        }
-        mma_commit_elect(s_full);
-      };
-      auto issue_dp = [&](int t) {   // dP^T = V dO_t^T
-        const uint32_t v_lo = lo(L::V_OFF, kKM), do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kKM);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
-          mma_ss_elect(tmem + L::DPT_COL, sdesc_join(v_lo + off, kHi), sdesc_join(do_lo + off, kHi), kIdS,
-                      kk > 0 ? 1u : 0u);
-        }
-        mma_commit_elect(dp_full);
-      };
-      bool ok = warp_wait(kv_full, 0, wc) && warp_wait(&q_full[0], 0, wc);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        ok = warp_wait(&do_full[0], 0, wc);
-        if (ok) {
-          tc_fence_after();
-          issue_dp(0);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
+        mma_ss_elect(tmem + L::ST_COL, sdesc_join(k_lo + off, kHi), sdesc_join(q_lo + off, kHi), kIdS,
+                    kk > 0 ? 1u : 0u);
       }
-      for (int t = 0; ok && t < n_iter; ++t) {
-        const bool more = t + 1 < n_iter;
+      mma_commit_elect(s_full);
+    };
+    auto issue_dp = [&](int g) {   // dP^T = V dO_g^T
+      const uint32_t v_lo = lo(L::V_OFF, kKM), do_lo = lo(L::DO_OFF + (g % DS) * L::TILE, kKM);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
+        mma_ss_elect(tmem + L::DPT_COL, sdesc_join(v_lo + off, kHi), sdesc_join(do_lo + off, kHi), kIdS,
+                    kk > 0 ? 1u : 0u);
+      }
+      mma_commit_elect(dp_full);
+    };
+    auto wait = [&](uint64_t* bar, uint32_t parity) { return warp_wait(bar, parity, wc); };
+    int g = 0, gi = 0;
+    bool ok = true;
+    for (int n = 0; ok; ++n) {
+      int id;
+      if (!queue.peek(n, id, wc)) { ok = false; break; }
+      queue.release(n, lane);
+      if (id < 0) break;
+      const BwdItem it = bwd_item(p, id);
+      if (!wait(kv_full, gi & 1)) { ok = false; break; }
+      // first S and dP of the item; dP overwrites the columns where the previous tile's dQ^T sat
+      if (!wait(&q_full[g % QS], (g / QS) & 1)) { ok = false; break; }
+      tc_fence_after();
+      issue_s(g);
+      if (g >= 1 && !wait(dq_empty, (g - 1) & 1)) { ok = false; break; }
+      if (!wait(&do_full[g % DS], (g / DS) & 1)) { ok = false; break; }
+      tc_fence_after();
+      issue_dp(g);
+      for (int t = 0; t < it.n_iter; ++t, ++g) {
+        const bool more = t + 1 < it.n_iter;
         const uint32_t acc0 = t > 0 ? 1u : 0u;
-        // dV += (P*Z)^T dO_t, query half by query half (A = (P*Z)^T in TMEM: half h packed at
-        // columns [64h, 64h+32); B = dO MN-major: N = D, K = 16 queries per step)
+        // dV += (P*Z)^T dO_g, query half by query half (A = (P*Z)^T in TMEM: half h packed at
+        // columns [64h, 64h+32); B = dO MN-major: N = D, K = 16 queries per step).  The compute
+        // warps give P of an item's first tile only after their dV epilogue of the previous item.
         {
-          const uint32_t do_lo = lo(L::DO_OFF + (t % DS) * L::TILE, kMN);
+          const uint32_t do_lo = lo(L::DO_OFF + (g % DS) * L::TILE, kMN);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!warp_wait(&p_full[h], t & 1, wc)) { ok = false; break; }
+            if (!wait(&p_full[h], g & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
@@ -428,20 +568,23 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           if (!ok) break;
         }
-        mma_commit_elect(&do_empty[t % DS]);   // dO_t: last read by dV_t
-        // S_{t+1} over the (P*Z)^T that dV_t has just been given
+        mma_commit_elect(&do_empty[g % DS]);   // dO_g: last read by dV_g
+        // S_{g+1} over the (P*Z)^T that dV_g has just been given
         if (more) {
-          if (!warp_wait(&q_full[(t + 1) % QS], ((t + 1) / QS) & 1, wc)) { ok = false; break; }
+          if (!wait(&q_full[(g + 1) % QS], ((g + 1) / QS) & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_s(t + 1);
+          issue_s(g + 1);
         }
-        // dK += dS^T Q_t, query half by query half (A = dS^T in TMEM over the dP^T columns, half h
+        // the first dK of an item overwrites the accumulator: the previous item's dK epilogue must
+        // have read it
+        if (t == 0 && gi >= 1 && !wait(dk_free, (gi - 1) & 1)) { ok = false; break; }
+        // dK += dS^T Q_g, query half by query half (A = dS^T in TMEM over the dP^T columns, half h
         // packed at [128 + 64h, 128 + 64h + 32); B = Q MN-major)
         {
-          const uint32_t q_lo = lo(L::Q_OFF + (t % QS) * L::TILE, kMN);
+          const uint32_t q_lo = lo(L::Q_OFF + (g % QS) * L::TILE, kMN);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            if (!warp_wait(&ds_full[h], t & 1, wc)) { ok = false; break; }
+            if (!wait(&ds_full[h], g & 1)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
@@ -450,8 +593,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           if (!ok) break;
         }
-        mma_commit_elect(&q_empty[t % QS]);    // Q_t: last read by dK_t
-        // dQ^T = K^T dS^T over the dS^T/dP^T columns, after dK_t has read them
+        mma_commit_elect(&q_empty[g % QS]);    // Q_g: last read by dK_g
+        // dQ^T = K^T dS^T over the dS^T/dP^T columns, after dK_g has read them
         // (M = D, N = 128 queries, K = 128 keys; B = dS^T from shared memory)
         {
           const uint32_t k_lo = lo(L::K_OFF, kMN), ds_lo = lo(L::DS_OFF, kMN);
@@ -462,17 +605,23 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         mma_commit_elect(dq_full);
         mma_commit_elect(ds_free);             // the shared-memory dS tile is free again
-        // dP_{t+1} once the dQ warps have read dQ^T out of those columns
+        // dP_{g+1} once the dQ warps have read dQ^T out of those columns
         if (more) {
-          if (!warp_wait(dq_empty, t & 1, wc)) { ok = false; break; }
-          if (!warp_wait(&do_full[(t + 1) % DS], ((t + 1) / DS) & 1, wc)) { ok = false; break; }
+          if (!wait(dq_empty, g & 1)) { ok = false; break; }
+          if (!wait(&do_full[(g + 1) % DS], ((g + 1) / DS) & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_dp(t + 1);
+          issue_dp(g + 1);
         }
       }
-      mma_commit_elect(fin);
-      if (lane == 0) mbar_drain(fin, 0, p.wait_ns);
+      if (!ok) break;
+      mma_commit_elect(fin);        // the item's dV and dK are complete
+      mma_commit_elect(kv_empty);   // and K, V are no longer read
+      ++gi;
     }
+    // every MMA issued above completes before TMEM is released: wait for the last item's fin (on
+    // an abort, commit once more and wait for that)
+    if (!ok) mma_commit_elect(fin);
+    if (lane == 0 && (gi >= 1 || !ok)) mbar_drain(fin, ok ? ((gi - 1) & 1) : (gi & 1), p.wait_ns);
     __syncwarp();
   } else if (warp < 8) {
     // =========================================================== compute (key row r, query half qh)
@@ -480,26 +629,35 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int qh = warp >> 2;                 // query columns [64 qh, 64 qh + 64) of every tile
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int key = k0 + r;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
     uint8_t* ds_smem = smem + L::DS_OFF + qh * L::SUB;   // this half's 64 query columns: one panel
-    for (int t = 0; t < n_iter; ++t) {
-      const int sq = t % QS;
+    int g = 0, gi = 0;   // query tiles and items with tiles so far (barrier phases)
+    for (int n = 0; ok; ++n) {   // items of the queue
+    int id;
+    if (!queue.peek(n, id, wc)) { ok = false; break; }
+    queue.release(n, lane);
+    if (id < 0) break;
+    const BwdItem itm = bwd_item(p, id);
+    const int kt = itm.kt, k0 = itm.k0, kv_end = itm.kv_end, q_first = itm.q_first, n_iter = itm.n_iter;
+    const uint64_t row_base = itm.row_base;
+    const int key = k0 + r;
+    for (int t = 0; t < n_iter; ++t, ++g) {   // (body indented one level less than the loop above)
+      const int sq = g % QS;
       const int qrow0 = (q_first + t) * 128;
       const int qc0 = qrow0 + 64 * qh;         // first query of this half
       const float* st_l = stat + sq * 256 + 64 * qh;
       const bool need_mask = (k0 + 128 > kv_end) || (qc0 + 64 > p.N) || (p.causal && q_first + t == kt);
       uint32_t kb[2] = {0u, 0u};   // dropout keep bits of this key row: query 64 qh + c -> bit c % 32 of kb[c / 32]
       if (DROPOUT) {
-        if (!warp_wait(&keep_full[t & 1], (t >> 1) & 1, wc)) { ok = false; break; }
-        const uint2 w = reinterpret_cast<const uint2*>(&keep_smem[(t & 1) * 128 + r])[qh];
+        if (!warp_wait(&keep_full[g & 1], (g >> 1) & 1, wc)) { ok = false; break; }
+        const uint2 w = reinterpret_cast<const uint2*>(&keep_smem[(g & 1) * 128 + r])[qh];
         kb[0] = w.x;
         kb[1] = w.y;
       }
-      if (!warp_wait(s_full, t & 1, wc)) { ok = false; break; }
-      if (!warp_wait(&stat_full[sq], (t / QS) & 1, wc)) { ok = false; break; }
+      if (!warp_wait(s_full, g & 1, wc)) { ok = false; break; }
+      if (!warp_wait(&stat_full[sq], (g / QS) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       // ---- P^T = exp2(S^T tau log2e - lse2) over this half's 64 query columns
       float pr[64];
@@ -513,13 +671,18 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       }
       {
         const uint64_t sl2x2 = f2_make(sl2, sl2);
-        const uint64_t* nl2 = reinterpret_cast<const uint64_t*>(st_l);   // pairs of -lse2
+        // -lse2 of four query columns per 16-byte (broadcast) load
+        const float4* nl4 = reinterpret_cast<const float4*>(st_l);
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float x0, x1;
-          f2_split(f2_fma(f2_make(pr[c], pr[c + 1]), sl2x2, nl2[c >> 1]), x0, x1);
+        for (int c = 0; c < 64; c += 4) {
+          const float4 nl = nl4[c >> 2];
+          float x0, x1, x2, x3;
+          f2_split(f2_fma(f2_make(pr[c], pr[c + 1]), sl2x2, f2_make(nl.x, nl.y)), x0, x1);
+          f2_split(f2_fma(f2_make(pr[c + 2], pr[c + 3]), sl2x2, f2_make(nl.z, nl.w)), x2, x3);
           pr[c] = ex2_approx(x0);
           pr[c + 1] = ex2_approx(x1);
+          pr[c + 2] = ex2_approx(x2);
+          pr[c + 3] = ex2_approx(x3);
         }
       }
       if (need_mask) {
@@ -554,15 +717,15 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // ---- dS^T = P^T * (dP^T Z/(1-p) - D), in chunks of 32 query columns; written twice: as bf16
       // pairs into TMEM over the dP^T columns already read (the A operand of dK) and into this
       // half's shared-memory panel (the B operand of dQ^T)
-      if (!warp_wait(dp_full, t & 1, wc)) { ok = false; break; }
-      // the shared-memory dS tile is free: dQ^T_{t-1} has read it
-      if (t >= 1 && !warp_wait(ds_free, (t - 1) & 1, wc)) { ok = false; break; }
+      if (!warp_wait(dp_full, g & 1, wc)) { ok = false; break; }
+      // the shared-memory dS tile is free: dQ^T of the previous tile has read it
+      if (g >= 1 && !warp_wait(ds_free, (g - 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       if (DROPOUT) {
         // The keep bits again, through a volatile read: otherwise the compiler keeps the per-column
         // keep predicates of the P phase alive across the dP wait, which costs registers (spills).
         const volatile uint32_t* kv =
-            reinterpret_cast<const volatile uint32_t*>(&keep_smem[(t & 1) * 128 + r]) + 2 * qh;
+            reinterpret_cast<const volatile uint32_t*>(&keep_smem[(g & 1) * 128 + r]) + 2 * qh;
         kb[0] = kv[0];
         kb[1] = kv[1];
       }
@@ -573,10 +736,11 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_ld_wait();
         reg_fence32(dr);
         uint32_t pk[16];
-        const uint64_t* nd2 = reinterpret_cast<const uint64_t*>(st_l + 128);   // pairs of -D
+        const float4* nd4 = reinterpret_cast<const float4*>(st_l + 128);   // -D, four columns per load
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = 32 * cc + 2 * e;
+          const float4 nd = nd4[c >> 2];
           float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
           if (DROPOUT) {
             const uint32_t kbits = kb[cc];
@@ -584,7 +748,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             dpb = ((kbits >> ((c + 1) & 31)) & 1u) ? dpb * p.drop_scale : 0.f;
           }
           float da, db;   // dS = P (dP - D), as P * (dP + (-D)) on pairs
-          f2_split(f2_mul(f2_make(pr[c], pr[c + 1]), f2_add(f2_make(dpa, dpb), nd2[c >> 1])), da, db);
+          const uint64_t nd2 = (e & 1) ? f2_make(nd.z, nd.w) : f2_make(nd.x, nd.y);
+          f2_split(f2_mul(f2_make(pr[c], pr[c + 1]), f2_add(f2_make(dpa, dpb), nd2)), da, db);
           pk[e] = pack_bf16x2(da, db);
         }
         tmem_st16(lane_base + L::DPT_COL + 64 * qh + 16 * cc, pk);
@@ -602,16 +767,13 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[qh]);
     }
+    if (!ok) break;
     // ---- dV epilogue: this half of the feature columns
     constexpr int HD = D / 2;
-    if (n_iter == 0) {
-      if (key < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dv + (row_base + key) * D + qh * HD);
-#pragma unroll
-        for (int c = 0; c < HD / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-      }
-    } else if (ok && warp_wait(fin, 0, wc)) {
-      tc_fence_after();
+    if (!warp_wait(fin, gi & 1, wc)) { ok = false; break; }
+    ++gi;
+    tc_fence_after();
+    {
       const float s = DROPOUT ? p.drop_scale : 1.f;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
@@ -621,6 +783,10 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         reg_fence32(vr);
         if (key < p.N) store_row32(p.dv + (row_base + key) * D + qh * HD + c * 32, vr, s, p.out_align32);
       }
+    }
+    // the next item's first dV MMA (which overwrites the accumulator) waits for this warp's next
+    // P arrival, which comes after these reads
+    tc_fence_before();
     }
   } else {
     // =========================================================== dQ + dK epilogue (warps 8-11)
@@ -639,60 +805,70 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float* stage = reinterpret_cast<float*>(smem + L::STG_OFF + quarter * L::STAGE_BYTES);
     const bool lane_ok = lane < L::FPW;
     bool ok = true;
-    if (DROPOUT) {   // keep bits of the first two tiles
-      for (int t = 0; t < 2 && t < n_iter; ++t) {
-        keep_smem[t * 128 + r] = keep_bits_row(p, row_base, (q_first + t) * 128, k0 + r);
+    // dropout: keep bits of the tiles ahead, walking this CTA's tiles (they may belong to later items)
+    BwdTileCursor ahead;
+    if (DROPOUT) {
+      ok = ahead.start(p, queue, wc);
+      for (int s2 = 0; ok && s2 < 2 && ahead.valid; ++s2) {   // the first two tiles
+        keep_smem[s2 * 128 + r] =
+            keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0 + r);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&keep_full[t]);
+        if (lane == 0) mbar_arrive(&keep_full[s2]);
+        ok = ahead.advance(p, queue, wc);
       }
     }
-    for (int t = 0; t < n_iter; ++t) {
-      const int qrow0 = (q_first + t) * 128;
-      if (!warp_wait(dq_full, t & 1, wc)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t g[128];
+    int g = 0, gi = 0;   // query tiles and items with tiles so far (barrier phases)
+    for (int n = 0; ok; ++n) {
+      int id;
+      if (!queue.peek(n, id, wc)) { ok = false; break; }
+      queue.release(n, lane);
+      if (id < 0) break;
+      const BwdItem itm = bwd_item(p, id);
+      const int key = itm.k0 + r;
+      for (int t = 0; t < itm.n_iter; ++t, ++g) {
+        const int qrow0 = (itm.q_first + t) * 128;
+        if (!warp_wait(dq_full, g & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t gq[128];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(lane_base + L::DPT_COL + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&g[32 * c]));
-      tmem_ld_wait();
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(lane_base + L::DPT_COL + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&gq[32 * c]));
+        tmem_ld_wait();
 #pragma unroll
-      for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&g[h * 32]));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_empty);
-#pragma unroll
-      for (int rd = 0; rd < L::ROUNDS; ++rd) {
-        // the previous reduction from this staging slice must have read it
-        if (lane == 0) bulk_wait_read0();
+        for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&gq[h * 32]));
+        tc_fence_before();
         __syncwarp();
-        if (lane_ok) {
+        if (lane == 0) mbar_arrive(dq_empty);
 #pragma unroll
-          for (int c = 0; c < L::QPR; ++c) stage[c * L::FPW + lane] = __uint_as_float(g[rd * L::QPR + c]);
+        for (int rd = 0; rd < L::ROUNDS; ++rd) {
+          // the previous reduction from this staging slice must have read it
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          if (lane_ok) {
+#pragma unroll
+            for (int c = 0; c < L::QPR; ++c) stage[c * L::FPW + lane] = __uint_as_float(gq[rd * L::QPR + c]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {   // rows past N are outside the tensor map and are not written
+            tma_reduce_add_3d(&tm_dq, stage, quarter * L::FPW, qrow0 + rd * L::QPR, itm.bh);
+            bulk_commit();
+          }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {   // rows past N are outside the tensor map and are not written
-          tma_reduce_add_3d(&tm_dq, stage, quarter * L::FPW, qrow0 + rd * L::QPR, bh);
-          bulk_commit();
+        // the compute warps have finished tile g (dq_full follows ds_full): its keep-bit stage is
+        // free for the tile two ahead
+        if (DROPOUT && ahead.valid) {
+          keep_smem[(g & 1) * 128 + r] =
+              keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0 + r);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&keep_full[g & 1]);
+          if (!ahead.advance(p, queue, wc)) { ok = false; break; }
         }
       }
-      // the compute warps have finished tile t (dq_full follows ds_full): its keep-bit stage is free
-      if (DROPOUT && t + 2 < n_iter) {
-        keep_smem[(t & 1) * 128 + r] = keep_bits_row(p, row_base, (q_first + t + 2) * 128, k0 + r);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&keep_full[t & 1]);
-      }
-    }
-    if (lane == 0) bulk_wait0();   // every reduction has completed before the kernel ends
-    __syncwarp();
-    const int key = k0 + r;
-    if (n_iter == 0) {
-      if (key < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dk + (row_base + key) * D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-      }
-    } else if (ok && warp_wait(fin, 0, wc)) {
+      if (!ok) break;
+      // ---- dK epilogue
+      if (!warp_wait(fin, gi & 1, wc)) { ok = false; break; }
+      ++gi;
       tc_fence_after();
       const float s = p.scale;
 #pragma unroll
@@ -701,9 +877,15 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tmem_ld32(lane_base + L::DK_COL + c * 32, kr);
         tmem_ld_wait();
         reg_fence32(kr);
-        if (key < p.N) store_row32(p.dk + (row_base + key) * D + c * 32, kr, s, p.out_align32);
+        if (key < p.N) store_row32(p.dk + (itm.row_base + key) * D + c * 32, kr, s, p.out_align32);
       }
+      // the accumulator has been read: the next item's first dK may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dk_free);
     }
+    if (lane == 0) bulk_wait0();   // every reduction has completed before the kernel ends
+    __syncwarp();
   }
 
   tc_fence_before();

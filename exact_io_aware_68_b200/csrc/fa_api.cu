@@ -15,6 +15,7 @@
 #include "../../include/fa.h"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
+#include "fwd256_sm100.cuh"
 #include "fwd_sm100.cuh"
 #include "simt_f32.cuh"
 
@@ -90,13 +91,18 @@ fa_status make_dq_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, u
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-fa_status check_common(int B, int H, int N, int d, float scale, float dropout_p, bool bf16) {
+// Which head dimensions an entry point takes.
+enum class Dims { kBf16, kBf16Fwd, kF32 };
+
+fa_status check_common(int B, int H, int N, int d, float scale, float dropout_p, Dims dims) {
   if (B < 1 || H < 1 || N < 1) return fail(FA_ERR_INVALID_ARG, "B, H and N must be >= 1 (got %d, %d, %d)", B, H, N);
   if (int64_t(B) * H > 65535) return fail(FA_ERR_UNSUPPORTED, "B*H = %lld exceeds 65535", (long long)B * H);
   if (int64_t(N) > (int64_t(1) << 30)) return fail(FA_ERR_UNSUPPORTED, "N = %d is too large", N);
-  if (bf16 && d != 64 && d != 128)
-    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: bf16 supports d in {64, 128}", d);
-  if (!bf16 && (d < 1 || d > 128))
+  if (dims == Dims::kBf16 && d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: this bf16 entry point supports d in {64, 128}", d);
+  if (dims == Dims::kBf16Fwd && d != 64 && d != 128 && d != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: the bf16 forward supports d in {64, 128, 256}", d);
+  if (dims == Dims::kF32 && (d < 1 || d > 128))
     return fail(FA_ERR_UNSUPPORTED, "head dimension d = %d: fp32 supports 1 <= d <= 128", d);
   if (!std::isfinite(scale) || !(scale > 0.f)) return fail(FA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (!(dropout_p >= 0.f) || !(dropout_p < 1.f)) return fail(FA_ERR_INVALID_ARG, "dropout_p must be in [0, 1)");
@@ -123,13 +129,14 @@ uint32_t drop_threshold(float p) {
 struct Workspace {
   float* dq_acc;
   float* dvec;
+  unsigned int* work_ctr;
 };
 size_t ws_dq_bytes(int B, int H, int N, int d) {
   return (size_t(B) * H * N * d * 4 + 255) & ~size_t(255);
 }
-size_t ws_total_bytes(int B, int H, int N, int d) {
-  return ws_dq_bytes(B, H, N, d) + ((size_t(B) * H * N * 4 + 255) & ~size_t(255));
-}
+size_t ws_d_bytes(int B, int H, int N) { return (size_t(B) * H * N * 4 + 255) & ~size_t(255); }
+// fp32 dQ accumulator, D, and 256 bytes for the main kernel's item counter
+size_t ws_total_bytes(int B, int H, int N, int d) { return ws_dq_bytes(B, H, N, d) + ws_d_bytes(B, H, N) + 256; }
 fa_status check_workspace(void* ws, size_t bytes, int B, int H, int N, int d, Workspace* out) {
   if (ws == nullptr) return fail(FA_ERR_INVALID_ARG, "workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(FA_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
@@ -137,6 +144,8 @@ fa_status check_workspace(void* ws, size_t bytes, int B, int H, int N, int d, Wo
   if (bytes < need) return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", bytes, need);
   out->dq_acc = static_cast<float*>(ws);
   out->dvec = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_dq_bytes(B, H, N, d));
+  out->work_ctr =
+      reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + ws_dq_bytes(B, H, N, d) + ws_d_bytes(B, H, N));
   return FA_OK;
 }
 
@@ -227,12 +236,12 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
     return st;
   int sms = 0;
   if ((st = sm_count(&sms)) != FA_OK) return st;
-  // Blocks are dispatched in linear order. Head-major order (x = key tile, y = head) keeps the
-  // CTAs in flight on a few heads, so their Q and dO stay in L2, but each head's heaviest causal
-  // CTA starts only when the head does. That tail is about 2 * SMs / (B*H*n_tiles) of the run.
-  // While the grid has at most 20 CTAs per SM, a 1-D grid is used instead: groups of heads one
-  // after another, key-tile-major inside each group. Every head's first key tile (the most query
-  // tiles when causal) then starts with its group, and the one-tile CTAs form each group's tail.
+  // Items (head, key tile) are taken in a linear launch order. Head-major order keeps the CTAs
+  // in flight on a few heads, so their Q and dO stay in L2, but each head's heaviest causal key
+  // tile starts only when the head does. That tail is about 2 * SMs / (B*H*n_tiles) of the run.
+  // While there are at most 20 items per SM, the order is instead: groups of heads one after
+  // another, key-tile-major inside each group. Every head's first key tile (the most query
+  // tiles when causal) then starts with its group, and the one-tile items form each group's tail.
   // A group holds at most 16 heads, and its Q, dO and fp32 dQ accumulator (8*N*d bytes a head)
   // fit in 32 MB of L2. Measured on the headline causal 2x16x4096x128: head-major 352 us,
   // key-tile-major over all 32 heads 332-340 us (2.6x the algorithmic DRAM bytes), groups of 8
@@ -242,7 +251,10 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   size_t l2 = 0;
   if ((st = l2_bytes(&l2)) != FA_OK) return st;
   p.head_group = fa_bwd_head_group(p.N, D, l2);
-  const dim3 grid = p.kt_major ? dim3(unsigned(p.B * p.H * p.n_tiles)) : dim3(p.n_tiles, p.B * p.H);
+  // persistent: one CTA per SM (or fewer when there are fewer items), each walking items
+  // c, c + G, c + 2G, ... of the launch order
+  const long long items = (long long)p.B * p.H * p.n_tiles;
+  const dim3 grid(unsigned(items < sms ? items : sms));
   fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, fa::kBwdThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status("fa_bwd main kernel launch");
 }
@@ -253,6 +265,7 @@ fa::BwdParams bwd_params(int B, int H, int N, float scale, int causal, const int
   p.lse = nullptr;
   p.dvec = w.dvec;
   p.dq_acc = w.dq_acc;
+  p.work_ctr = w.work_ctr;
   p.key_lens = key_lens;
   p.B = B;
   p.H = H;
@@ -305,6 +318,44 @@ fa_status launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   return launch_status("fa_fwd_decode combine kernel launch");
 }
 
+// The d = 256 forward (fwd256_sm100.cuh): one query tile per CTA, 64-key blocks, persistent grid.
+fa_status fwd256(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, float scale,
+                 int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t s) {
+  using L = fa::Fwd256Layout;
+  CUtensorMap mq, mk, mv;
+  fa_status st;
+  if ((st = make_tile_map(&mq, q, B * H, N, 256, "q")) != FA_OK) return st;
+  if ((st = make_tile_map(&mk, k, B * H, N, 256, "k", 64)) != FA_OK) return st;
+  if ((st = make_tile_map(&mv, v, B * H, N, 256, "v", 64)) != FA_OK) return st;
+  fa::Fwd256Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.key_lens = key_lens;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.n_qtiles = (N + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.dropout = dropout_p > 0.f ? 1 : 0;
+  p.drop_thr = drop_threshold(dropout_p);
+  p.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
+  p.seed = seed;
+  p.wait_ns = g_wait_ns.load();
+  int sms = 0;
+  if ((st = sm_count(&sms)) != FA_OK) return st;
+  const long long items = (long long)p.n_qtiles * B * H;
+  const dim3 grid(unsigned(items < sms ? items : sms));
+  if (p.dropout) {
+    if ((st = set_smem(fa::fa_fwd256_sm100_kernel<true>, L::BYTES)) != FA_OK) return st;
+    fa::fa_fwd256_sm100_kernel<true><<<grid, 256, L::BYTES, s>>>(mq, mk, mv, p);
+  } else {
+    if ((st = set_smem(fa::fa_fwd256_sm100_kernel<false>, L::BYTES)) != FA_OK) return st;
+    fa::fa_fwd256_sm100_kernel<false><<<grid, 256, L::BYTES, s>>>(mq, mk, mv, p);
+  }
+  return launch_status("fa_fwd (d = 256) kernel launch");
+}
+
 unsigned grid_for(uint64_t work, unsigned per_block) {
   const uint64_t g = (work + per_block - 1) / per_block;
   return unsigned(g < 1 ? 1 : (g > (1u << 30) ? (1u << 30) : g));
@@ -326,13 +377,14 @@ int fa_bwd_head_group(int N, int d, size_t l2_bytes) {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream) {
-  fa_status st = check_common(B, H, N, d, scale, dropout_p, true);
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, Dims::kBf16Fwd);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(q);
   FA_CHECK_PTR(k);
   FA_CHECK_PTR(v);
   FA_CHECK_PTR(o);
   FA_CHECK_PTR(lse);
+  if (d == 256) return fwd256(q, k, v, o, lse, B, H, N, scale, causal, key_lens, dropout_p, seed, stream);
   CUtensorMap mq, mk, mv;
   if ((st = make_tile_map(&mq, q, B * H, N, d, "q")) != FA_OK) return st;
   if ((st = make_tile_map(&mk, k, B * H, N, d, "k")) != FA_OK) return st;
@@ -362,7 +414,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 fa_status fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
                      float scale, int causal, const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream) {
-  fa_status st = check_common(B, H, N, d, scale, dropout_p, false);
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, Dims::kF32);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(q);
   FA_CHECK_PTR(k);
@@ -406,7 +458,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 
 fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream) {
-  fa_status st = check_common(B, H, N, d, 1.f, 0.f, true);
+  fa_status st = check_common(B, H, N, d, 1.f, 0.f, Dims::kBf16);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(o);
   FA_CHECK_PTR(dO);
@@ -427,7 +479,7 @@ fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d,
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
                       int B, int H, int N, int d, float scale, int causal, const int32_t* key_lens, float dropout_p,
                       uint64_t seed, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  fa_status st = check_common(B, H, N, d, scale, dropout_p, true);
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, Dims::kBf16);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(q);
   FA_CHECK_PTR(k);
@@ -458,7 +510,7 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* 
 
 fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream) {
-  fa_status st = check_common(B, H, N, d, scale, 0.f, true);
+  fa_status st = check_common(B, H, N, d, scale, 0.f, Dims::kBf16);
   if (st != FA_OK) return st;
   FA_CHECK_PTR(dq);
   Workspace w;
@@ -498,7 +550,7 @@ size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nkv, int d) {
 fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
                         int Nkv, int d, float scale, int causal, const int32_t* key_lens, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
-  fa_status st = check_common(B, H, Nkv, d, scale, 0.f, true);
+  fa_status st = check_common(B, H, Nkv, d, scale, 0.f, Dims::kBf16);
   if (st != FA_OK) return st;
   if (Nq < 1 || Nq > 64) return fail(FA_ERR_UNSUPPORTED, "Nq = %d: fa_fwd_decode takes 1 <= Nq <= 64", Nq);
   FA_CHECK_PTR(q);

@@ -26,8 +26,8 @@
  *  - Pointers are DEVICE pointers owned by the caller, 16-byte aligned; the library never
  *    allocates or frees device memory.  Outputs are overwritten, not accumulated.
  *  - scale (tau) must be finite and > 0 (1/sqrt(d) is the usual value).
- *  - bf16 entry points support d in {64, 128}, fa_fwd_f32 any 1 <= d <= 128; N >= 1 is arbitrary
- *    (tails are zero-filled by the tile loads and masked); B*H <= 65535.
+ *  - bf16 entry points support d in {64, 128} (fa_fwd also d = 256), fa_fwd_f32 any 1 <= d <= 128;
+ *    N >= 1 is arbitrary (tails are zero-filled by the tile loads and masked); B*H <= 65535.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  The return value reports argument validation and launch errors only.  Errors
  *    found on the device (a bounded wait that ran out) are reported by fa_check().
@@ -68,7 +68,7 @@ typedef enum {
 /* Forward, bf16 ("48 FlashAttention", block "Tiling и online softmax": tile by tile with a running
  * row max m and row sum l, O re-expressed when m moves; the operation of "FlashAttention 的第一原则",
  * section 2).  Writes o (bf16 [B,H,N,d]) and lse (fp32 [B,H,N]).  q, k, v: bf16 [B,H,N,d].
- * d in {64, 128}.  One kernel launch. */
+ * d in {64, 128, 256} (d = 256 has no backward).  One kernel launch. */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int H, int N, int d, float scale, int causal,
                  const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream);
@@ -79,8 +79,9 @@ FA_API fa_status fa_fwd_f32(const float* q, const float* k, const float* v, floa
                      int B, int H, int N, int d, float scale, int causal,
                      const int32_t* key_lens, float dropout_p, uint64_t seed, cudaStream_t stream);
 
-/* Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator [B,H,N,d] followed by
- * D = rowsum(dO * O) fp32 [B,H,N] (each part 256-byte aligned).  0 on invalid sizes. */
+/* Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator [B,H,N,d], D = rowsum(dO * O)
+ * fp32 [B,H,N] (each part 256-byte aligned) and 256 bytes for the main launch's work counter.
+ * 0 on invalid sizes. */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /* Backward, bf16 ("48 FlashAttention", block "Tiling и online softmax", paragraph "Backward — тоже
@@ -99,7 +100,8 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
 
 /* The three launches of fa_bwd, exposed separately (same arguments, same workspace) so that a
  * caller can time or interleave them.  Calling them in order is equivalent to fa_bwd.
- *  fa_bwd_prep:       D = rowsum(dO * O) into the workspace, clears the dQ accumulator.
+ *  fa_bwd_prep:       D = rowsum(dO * O) into the workspace, clears the dQ accumulator and the
+ *                     work counter (fa_bwd_main needs both cleared: run fa_bwd_prep before it).
  *  fa_bwd_main:       dK and dV (written), dQ accumulated (fp32) into the workspace.
  *  fa_bwd_dq_convert: dq = bf16(scale * accumulator). */
 FA_API fa_status fa_bwd_prep(const void* o, const void* dO, int B, int H, int N, int d,

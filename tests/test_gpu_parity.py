@@ -58,6 +58,24 @@ def test_forward_matches_oracle(w):
     assert l_err <= LSE_MAX_ABS, l_err
 
 
+FWD256_CASES = [wl(1, 2, 1, 256), wl(1, 2, 200, 256), wl(2, 1, 333, 256, causal=True),
+                wl(2, 2, 257, 256, causal=True, pad=(100, 257), p=0.1, seed=9), wl(1, 3, 1000, 256, pad=(1, 1000)),
+                wl(1, 2, 1024, 256, causal=True, factor=0.5)]
+
+
+@pytest.mark.parametrize("w", FWD256_CASES, ids=case_id)
+def test_forward_head_dim_256(w):
+    """The d = 256 forward (one query tile per CTA, 64-key blocks) against the oracle."""
+    x = make_inputs(w, with_do=False)
+    *_, o, lse = run_fwd(x)
+    O, L = oracle.forward(x["q64"], x["k64"], x["v64"], x["scale"], w.causal, x["key_lens"], w.dropout_p, x["seed"])
+    res = assert_o_close(to_f64(o), O, O_MAX_ABS_BF16, large_ok=True)
+    assert res["max_err_small"] <= O_MAX_ABS_BF16
+    l_err = float(np.abs(lse.cpu().numpy() - L).max())
+    print(f"{case_id(w)}: O max-abs {res['max_err']:.3e}, lse max-abs {l_err:.3e}")
+    assert l_err <= LSE_MAX_ABS, l_err
+
+
 def test_forward_fp32_path():
     w = wl(1, 1, 128, 64, dtype="f32", seed=0)
     x = make_inputs(w, with_do=False)

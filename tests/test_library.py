@@ -38,7 +38,7 @@ def test_version_and_workspace_size(lib):
     dq = B * H * N * d * 4
     dvec = B * H * N * 4
     size = lib.fa_bwd_workspace_size(B, H, N, d)
-    assert size == ((dq + 255) // 256) * 256 + ((dvec + 255) // 256) * 256
+    assert size == ((dq + 255) // 256) * 256 + ((dvec + 255) // 256) * 256 + 256   # + the work counter
     assert lib.fa_bwd_workspace_size(0, 1, 1, 64) == 0
     # ragged N keeps the second part 256-byte aligned
     assert lib.fa_bwd_workspace_size(1, 1, 3, 64) % 256 == 0
@@ -48,7 +48,7 @@ def test_version_and_workspace_size(lib):
     (dict(B=0), _lib.FA_ERR_INVALID_ARG),
     (dict(N=0), _lib.FA_ERR_INVALID_ARG),
     (dict(d=96), _lib.FA_ERR_UNSUPPORTED),
-    (dict(d=256), _lib.FA_ERR_UNSUPPORTED),
+    (dict(d=512), _lib.FA_ERR_UNSUPPORTED),
     (dict(scale=0.0), _lib.FA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), _lib.FA_ERR_INVALID_ARG),
     (dict(p=1.0), _lib.FA_ERR_INVALID_ARG),
@@ -74,6 +74,14 @@ def test_fp32_head_dim_range(lib, d, status):
     fake = 0x2000
     st = lib.fa_fwd_f32(fake, fake, fake, fake, fake, 1, 1, 16, d, 0.125, 0, None, 0.0, 0, None)
     assert st == status and b"fp32" in lib.fa_get_error()
+
+
+def test_backward_refuses_head_dim_256(lib):
+    """d = 256 has a forward only; every backward entry point refuses it before any device work."""
+    fake = 0x2000
+    st = lib.fa_bwd(fake, fake, fake, fake, fake, fake, fake, fake, fake, 1, 1, 128, 256, 0.0625, 0, None, 0.0, 0,
+                    0x10000, 1 << 30, None)
+    assert st == _lib.FA_ERR_UNSUPPORTED and b"256" in lib.fa_get_error()
 
 
 def test_bwd_workspace_validation(lib):
