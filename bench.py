@@ -179,20 +179,25 @@ def run_native(args, w, world, rank, local):
 
     def launches(tensors, events=None):
         qq, kk, vv, dd, oo, ll, gq, gk, gv = tensors
-        calls = [
-            ("fa_fwd", (qq, kk, vv, oo, ll, B, H, N, d, scale, causal, kl_ptr, p, seed, sp)),
-            ("fa_bwd_prep", (oo, dd, B, H, N, d, ws.data_ptr(), ws.numel(), sp)),
-            ("fa_bwd_main", (qq, kk, vv, ll, dd, gk, gv, B, H, N, d, scale, causal, kl_ptr, p, seed,
-                             ws.data_ptr(), ws.numel(), sp)),
-            ("fa_bwd_dq_convert", (gq, B, H, N, d, scale, ws.data_ptr(), ws.numel(), sp)),
-        ]
+        calls = [("fa_fwd", (qq, kk, vv, oo, ll, B, H, N, d, scale, causal, kl_ptr, p, seed, sp))]
+        if args.separate_dq:   # dK, dV and dQ in separate passes: one ABI call, three launches
+            calls.append(("fa_bwd_split", (qq, kk, vv, oo, ll, dd, gq, gk, gv, B, H, N, d, scale, causal, kl_ptr, p,
+                                           seed, ws.data_ptr(), ws.numel(), sp)))
+        else:
+            calls += [
+                ("fa_bwd_prep", (oo, dd, B, H, N, d, ws.data_ptr(), ws.numel(), sp)),
+                ("fa_bwd_main", (qq, kk, vv, ll, dd, gk, gv, B, H, N, d, scale, causal, kl_ptr, p, seed,
+                                 ws.data_ptr(), ws.numel(), sp)),
+                ("fa_bwd_dq_convert", (gq, B, H, N, d, scale, ws.data_ptr(), ws.numel(), sp)),
+            ]
         for i, (name, a) in enumerate(calls):
             _lib.call(name, *a)
             if events is not None:
                 events[i + 1].record(stream)
 
     dev_tensors = tuple(t.data_ptr() for t in (q, k, v, do, o, lse, dq, dk, dv))
-    names = ["fa_fwd", "fa_bwd_prep", "fa_bwd_main", "fa_bwd_dq_convert"]
+    names = ["fa_fwd", "fa_bwd_split"] if args.separate_dq else ["fa_fwd", "fa_bwd_prep", "fa_bwd_main",
+                                                                   "fa_bwd_dq_convert"]
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -200,7 +205,7 @@ def run_native(args, w, world, rank, local):
     _lib.call("fa_check", sp)
 
     sampler = ClockSampler(local)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -219,7 +224,7 @@ def run_native(args, w, world, rank, local):
     for s in range(args.steps):
         for i, n in enumerate(names):
             per_kernel[n].append(ev[s][i].elapsed_time(ev[s][i + 1]))
-        step_ms.append(ev[s][0].elapsed_time(ev[s][4]))
+        step_ms.append(ev[s][0].elapsed_time(ev[s][len(names)]))
     fwd_ms_local = statistics.mean(per_kernel["fa_fwd"])
     step_ms_local = statistics.mean(step_ms)
 
@@ -280,7 +285,7 @@ def run_native(args, w, world, rank, local):
         return None
 
     pk = peaks()
-    kflops = {"fa_fwd": w.fwd_flops(), "fa_bwd_main": 2.5 * w.fwd_flops()}
+    kflops = {"fa_fwd": w.fwd_flops(), "fa_bwd_split" if args.separate_dq else "fa_bwd_main": 2.5 * w.fwd_flops()}
     kbytes = algorithmic_bytes(B, H, N, d)
     kernels = {}
     for n in names:
@@ -329,7 +334,7 @@ def run_native(args, w, world, rank, local):
         "kernels": kernels,
         "e2e": {"value": round(e2e_tflops, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 4 * args.steps,   # fused: fwd, prep, main, convert; split: fwd, prep, main, dQ pass
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -381,7 +386,9 @@ def algorithmic_bytes(B, H, N, d):
     return {"fa_fwd": 4 * 2 * e + 4 * rows,
             "fa_bwd_prep": 2 * 2 * e + 4 * e + 4 * rows,
             "fa_bwd_main": 6 * 2 * e + 2 * 4 * rows,
-            "fa_bwd_dq_convert": 4 * e + 2 * e}
+            "fa_bwd_dq_convert": 4 * e + 2 * e,
+            # the whole backward with dQ in its own pass: read Q, K, V, O, dO, lse; write dQ, dK, dV (+ D)
+            "fa_bwd_split": 8 * 2 * e + 2 * 4 * rows}
 
 
 # ----------------------------------------------------------------------------- oracle timing
@@ -574,6 +581,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-dq", action="store_true",
+                    help="backward through fa_bwd_split (dQ in a pass of its own) instead of the fused dQ")
     ap.add_argument("--decode", type=int, nargs=5, metavar=("B", "H", "NQ", "NKV", "D"),
                     help="time the decode-shaped forward instead (Nq rows against a cache of Nkv keys)")
     ap.add_argument("--decode-causal", type=int, default=1)

@@ -20,6 +20,7 @@ SIGNATURES = {
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P]),
     "fa_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P, _SZ, _P]),
+    "fa_bwd_split": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P, _SZ, _P]),
     "fa_bwd_prep": (_I, [_P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "fa_bwd_main": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P, _SZ, _P]),
     "fa_bwd_dq_convert": (_I, [_P, _I, _I, _I, _I, _F, _P, _SZ, _P]),

@@ -59,8 +59,8 @@ def bwd_workspace(B, H, N, d, device):
 
 
 def attention_bwd(q, k, v, o, lse, do, scale=None, causal=False, key_lens=None, dropout_p=0.0, seed=0,
-                  workspace=None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV of exact attention (``fa_bwd``)."""
+                  workspace=None, dq=None, dk=None, dv=None, separate_dq=False):
+    """dQ, dK, dV of exact attention (``fa_bwd``; ``fa_bwd_split`` with ``separate_dq``)."""
     B, H, N, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
         _check_tensor(name, t, torch.bfloat16, (B, H, N, d))
@@ -74,7 +74,8 @@ def attention_bwd(q, k, v, o, lse, do, scale=None, causal=False, key_lens=None, 
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     with torch.cuda.device(q.device):   # the library launches on the current device
-        _lib.call("fa_bwd", q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+        _lib.call("fa_bwd_split" if separate_dq else "fa_bwd", q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                  o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                   dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale, int(bool(causal)),
                   _ptr(key_lens), float(dropout_p), int(seed), workspace.data_ptr(), workspace.numel(), _stream(q))
     return dq, dk, dv

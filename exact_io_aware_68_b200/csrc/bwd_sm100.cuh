@@ -290,7 +290,9 @@ struct BwdTileCursor {
 // sequence, so the Q/dO rings, the statistics and the keep bits run on from one item into the next:
 // the next item's first Q and dO tiles load while the previous one finishes, and its K/V load as soon
 // as the previous item's last MMA has read K and V.
-template <int D, bool DROPOUT>
+// DQ: the kernel also forms dQ^T per tile and adds it into the fp32 accumulator (the fused path);
+// without it (the separate-pass path, fa_bwd_split) it makes dK and dV only, and dS stays in TMEM.
+template <int D, bool DROPOUT, bool DQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -545,7 +547,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (!wait(&q_full[g % QS], (g / QS) & 1)) { ok = false; break; }
       tc_fence_after();
       issue_s(g);
-      if (g >= 1 && !wait(dq_empty, (g - 1) & 1)) { ok = false; break; }
+      if (DQ && g >= 1 && !wait(dq_empty, (g - 1) & 1)) { ok = false; break; }
       if (!wait(&do_full[g % DS], (g / DS) & 1)) { ok = false; break; }
       tc_fence_after();
       issue_dp(g);
@@ -594,20 +596,21 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           if (!ok) break;
         }
         mma_commit_elect(&q_empty[g % QS]);    // Q_g: last read by dK_g
-        // dQ^T = K^T dS^T over the dS^T/dP^T columns, after dK_g has read them
-        // (M = D, N = 128 queries, K = 128 keys; B = dS^T from shared memory)
-        {
+        if (DQ) {
+          // dQ^T = K^T dS^T over the dS^T/dP^T columns, after dK_g has read them
+          // (M = D, N = 128 queries, K = 128 keys; B = dS^T from shared memory)
           const uint32_t k_lo = lo(L::K_OFF, kMN), ds_lo = lo(L::DS_OFF, kMN);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss_elect(tmem + L::DPT_COL, sdesc_join(k_lo + kk * (2048 >> 4), kHi),
                         sdesc_join(ds_lo + kk * (2048 >> 4), kHi), kIdQ, kk > 0 ? 1u : 0u);
+          mma_commit_elect(dq_full);
+          mma_commit_elect(ds_free);             // the shared-memory dS tile is free again
         }
-        mma_commit_elect(dq_full);
-        mma_commit_elect(ds_free);             // the shared-memory dS tile is free again
-        // dP_{g+1} once the dQ warps have read dQ^T out of those columns
+        // dP_{g+1} once the dQ warps have read dQ^T out of those columns (with DQ; without it, the
+        // dK MMAs issued above read dS^T there first: MMAs run in issue order)
         if (more) {
-          if (!wait(dq_empty, g & 1)) { ok = false; break; }
+          if (DQ && !wait(dq_empty, g & 1)) { ok = false; break; }
           if (!wait(&do_full[(g + 1) % DS], ((g + 1) / DS) & 1)) { ok = false; break; }
           tc_fence_after();
           issue_dp(g + 1);
@@ -719,7 +722,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       // half's shared-memory panel (the B operand of dQ^T)
       if (!warp_wait(dp_full, g & 1, wc)) { ok = false; break; }
       // the shared-memory dS tile is free: dQ^T of the previous tile has read it
-      if (g >= 1 && !warp_wait(ds_free, (g - 1) & 1, wc)) { ok = false; break; }
+      if (DQ && g >= 1 && !warp_wait(ds_free, (g - 1) & 1, wc)) { ok = false; break; }
       tc_fence_after();
       if (DROPOUT) {
         // The keep bits again, through a volatile read: otherwise the compiler keeps the per-column
@@ -754,14 +757,16 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         tmem_st16(lane_base + L::DPT_COL + 64 * qh + 16 * cc, pk);
         // dS (queries contiguous) into the 128-byte-swizzled panel: row = key r, 16-byte chunks of 8
+        if (DQ) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = 4 * cc + u;
-          uint4* dst = reinterpret_cast<uint4*>(ds_smem + r * 128 + ((chunk ^ (r & 7)) << 4));
-          *dst = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          for (int u = 0; u < 4; ++u) {
+            const int chunk = 4 * cc + u;
+            uint4* dst = reinterpret_cast<uint4*>(ds_smem + r * 128 + ((chunk ^ (r & 7)) << 4));
+            *dst = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          }
         }
       }
-      fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+      if (DQ) fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -827,6 +832,19 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int key = itm.k0 + r;
       for (int t = 0; t < itm.n_iter; ++t, ++g) {
         const int qrow0 = (itm.q_first + t) * 128;
+        if (!DQ) {   // only the keep bits: wait until the compute warps have finished tile g
+          if (DROPOUT) {
+            if (!warp_wait(&ds_full[0], g & 1, wc) || !warp_wait(&ds_full[1], g & 1, wc)) { ok = false; break; }
+            if (ahead.valid) {
+              keep_smem[(g & 1) * 128 + r] =
+                  keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0 + r);
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&keep_full[g & 1]);
+              if (!ahead.advance(p, queue, wc)) { ok = false; break; }
+            }
+          }
+          continue;
+        }
         if (!warp_wait(dq_full, g & 1, wc)) { ok = false; break; }
         tc_fence_after();
         uint32_t gq[128];

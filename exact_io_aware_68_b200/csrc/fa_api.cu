@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "bwd_dq_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd256_sm100.cuh"
@@ -223,16 +224,17 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return launch_status("fa_fwd kernel launch");
 }
 
-template <int D, bool DROPOUT>
+template <int D, bool DROPOUT, bool DQ>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
                           fa::BwdParams p, cudaStream_t s) {
   using L = fa::BwdLayout<D, DROPOUT>;
   CUtensorMap mdq;
   fa_status st0 = make_dq_map(&mdq, p.dq_acc, p.B * p.H, p.N, D, L::FPW, L::QPR);
   if (st0 != FA_OK) return st0;
-  fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D, DROPOUT>, L::BYTES);
+  fa_status st = set_smem(fa::fa_bwd_sm100_kernel<D, DROPOUT, DQ>, L::BYTES);
   if (st != FA_OK) return st;
-  if ((st = check_launch_regs(fa::fa_bwd_sm100_kernel<D, DROPOUT>, fa::kBwdLaunchRegs, "fa_bwd main kernel")) != FA_OK)
+  if ((st = check_launch_regs(fa::fa_bwd_sm100_kernel<D, DROPOUT, DQ>, fa::kBwdLaunchRegs, "fa_bwd main kernel")) !=
+      FA_OK)
     return st;
   int sms = 0;
   if ((st = sm_count(&sms)) != FA_OK) return st;
@@ -255,8 +257,18 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   // c, c + G, c + 2G, ... of the launch order
   const long long items = (long long)p.B * p.H * p.n_tiles;
   const dim3 grid(unsigned(items < sms ? items : sms));
-  fa::fa_bwd_sm100_kernel<D, DROPOUT><<<grid, fa::kBwdThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
+  fa::fa_bwd_sm100_kernel<D, DROPOUT, DQ><<<grid, fa::kBwdThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status("fa_bwd main kernel launch");
+}
+
+template <int D, bool DROPOUT>
+fa_status launch_dq_pass(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
+                         const fa::DqParams& p, dim3 grid, cudaStream_t s) {
+  using L = fa::DqLayout<D>;
+  const fa_status st = set_smem(fa::fa_bwd_dq_pass_kernel<D, DROPOUT>, L::BYTES);
+  if (st != FA_OK) return st;
+  fa::fa_bwd_dq_pass_kernel<D, DROPOUT><<<grid, 256, L::BYTES, s>>>(mq, mk, mv, mdo, p);
+  return launch_status("fa_bwd_split dQ kernel launch");
 }
 
 fa::BwdParams bwd_params(int B, int H, int N, float scale, int causal, const int32_t* key_lens, float dropout_p,
@@ -502,10 +514,74 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const float* 
   p.out_align32 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
   cudaStream_t s = stream;
   if (d == 64)
-    return p.dropout ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, s)
-                     : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, s);
-  return p.dropout ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, s)
-                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, s);
+    return p.dropout ? launch_bwd_main<64, true, true>(mq, mk, mv, mdo, p, s)
+                     : launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, s);
+  return p.dropout ? launch_bwd_main<128, true, true>(mq, mk, mv, mdo, p, s)
+                   : launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, s);
+}
+
+fa_status fa_bwd_split(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                       void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                       const int32_t* key_lens, float dropout_p, uint64_t seed, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  fa_status st = check_common(B, H, N, d, scale, dropout_p, Dims::kBf16);
+  if (st != FA_OK) return st;
+  FA_CHECK_PTR(q);
+  FA_CHECK_PTR(k);
+  FA_CHECK_PTR(v);
+  FA_CHECK_PTR(lse);
+  FA_CHECK_PTR(dO);
+  FA_CHECK_PTR(dq);
+  FA_CHECK_PTR(dk);
+  FA_CHECK_PTR(dv);
+  Workspace w;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d, &w)) != FA_OK) return st;
+  if ((st = fa_bwd_prep(o, dO, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_tile_map(&mq, q, B * H, N, d, "q")) != FA_OK) return st;
+  if ((st = make_tile_map(&mk, k, B * H, N, d, "k")) != FA_OK) return st;
+  if ((st = make_tile_map(&mv, v, B * H, N, d, "v")) != FA_OK) return st;
+  if ((st = make_tile_map(&mdo, dO, B * H, N, d, "dO")) != FA_OK) return st;
+  // dK and dV: the main kernel without its dQ part
+  fa::BwdParams p = bwd_params(B, H, N, scale, causal, key_lens, dropout_p, seed, w);
+  p.lse = lse;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.out_align32 = ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31u) == 0 ? 1 : 0;
+  if (d == 64)
+    st = p.dropout ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, stream)
+                   : launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, stream);
+  else
+    st = p.dropout ? launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, stream)
+                   : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, stream);
+  if (st != FA_OK) return st;
+  // dQ: its own pass, query-tile-major
+  fa::DqParams dp{};
+  dp.dq = static_cast<__nv_bfloat16*>(dq);
+  dp.lse = lse;
+  dp.dvec = w.dvec;
+  dp.key_lens = key_lens;
+  dp.B = B;
+  dp.H = H;
+  dp.N = N;
+  dp.n_qtiles = (N + 127) / 128;
+  dp.causal = causal ? 1 : 0;
+  dp.scale = scale;
+  dp.scale_log2 = scale * 1.4426950408889634f;
+  dp.dropout = dropout_p > 0.f ? 1 : 0;
+  dp.drop_thr = drop_threshold(dropout_p);
+  dp.drop_scale = dropout_p > 0.f ? 1.f / (1.f - dropout_p) : 1.f;
+  dp.seed = seed;
+  dp.wait_ns = g_wait_ns.load();
+  int sms = 0;
+  if ((st = sm_count(&sms)) != FA_OK) return st;
+  const long long items = (long long)dp.n_qtiles * B * H;
+  const dim3 grid(unsigned(items < sms ? items : sms));
+  if (d == 64)
+    return dp.dropout ? launch_dq_pass<64, true>(mq, mk, mv, mdo, dp, grid, stream)
+                      : launch_dq_pass<64, false>(mq, mk, mv, mdo, dp, grid, stream);
+  return dp.dropout ? launch_dq_pass<128, true>(mq, mk, mv, mdo, dp, grid, stream)
+                    : launch_dq_pass<128, false>(mq, mk, mv, mdo, dp, grid, stream);
 }
 
 fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,

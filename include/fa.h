@@ -113,6 +113,19 @@ FA_API fa_status fa_bwd_main(const void* q, const void* k, const void* v, const 
 FA_API fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Backward with dQ in a pass of its own: the same arguments and results as fa_bwd (same workspace).
+ * Three launches: fa_bwd_prep; the main kernel making dK and dV only; a query-tile-major kernel that
+ * recomputes S, P and dP per key block and accumulates dQ = scale * dS K in tensor memory, writing
+ * each dQ row once (no fp32 accumulator reductions).  It recomputes two of the five matmuls, so it
+ * does more arithmetic than fa_bwd; both are kept so that the two ways of forming dQ that the
+ * method allows ("48 FlashAttention", block "Tiling и online softmax": dQ accumulated atomically or
+ * in a separate pass) can be compared. */
+FA_API fa_status fa_bwd_split(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv,
+                       int B, int H, int N, int d, float scale, int causal,
+                       const int32_t* key_lens, float dropout_p, uint64_t seed,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Backward that allocates nothing, for callers that cannot allocate device memory: a plugin
  * inside another runtime that owns all device memory and hands it no workspace, or a
  * latency-critical loop that cannot afford cudaMalloc's implicit device synchronisation.
