@@ -27,6 +27,7 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _F, _U64, _P]),
     "fa_bwd_noalloc_max_scratch": (_SZ, []),
     "fa_fwd_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_fwd_decode_split": (_I, [_I, _I, _I, _I]),
     "fa_fwd_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _SZ, _P]),
     "fa_bwd_head_group": (_I, [_I, _I, _SZ]),
     "fa_dropout_mask": (_I, [_P, _I, _I, _I, _F, _U64, _P]),

@@ -35,8 +35,8 @@ struct DqLayout {
   static constexpr int V_OFF = K_OFF + KST * TILE;
   static constexpr int BAR_OFF = V_OFF + VST * TILE;
   // qd_full, qd_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], dp_full,
-  // dp_read, ds_full, dq_fin, dq_free, fin
-  static constexpr int NBARS = 2 + 2 * KST + 2 * VST + 2 + 6;
+  // dp_read, ds_full[2], dq_fin, dq_free, fin
+  static constexpr int NBARS = 2 + 2 * KST + 2 * VST + 2 + 7;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int DP_COL = 256, DQ_COL = 384;
@@ -85,8 +85,10 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   uint64_t* s_full = v_empty + VST;   // [2]: score buffer
   uint64_t* dp_full = s_full + 2;
   uint64_t* dp_read = dp_full + 1;    // the compute warps hold dP(j) in registers
+  // [2]: score buffer.  One per buffer, so that the compute warps cannot complete a barrier twice
+  // before the MMA warp has waited on it: block j + 2 needs S(j + 2), issued after dQ(j).
   uint64_t* ds_full = dp_read + 1;
-  uint64_t* dq_fin = ds_full + 1;     // per item
+  uint64_t* dq_fin = ds_full + 2;     // per item
   uint64_t* dq_free = dq_fin + 1;     // per item
   uint64_t* fin = dq_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
@@ -123,7 +125,8 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
     mbar_init(dp_read, 4);
-    mbar_init(ds_full, 4);
+    mbar_init(&ds_full[0], 4);
+    mbar_init(&ds_full[1], 4);
     mbar_init(dq_fin, 1);
     mbar_init(dq_free, 4);
     mbar_init(fin, 1);
@@ -233,7 +236,7 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         // dQ += dS(j) K_j   (A = dS in TMEM: 16 keys per step = 8 packed columns; B = K_j MN-major)
         if (j == 0 && ni >= 1 && !wait(dq_free, (ni - 1) & 1)) { ok = false; break; }
-        if (!wait(ds_full, b & 1)) { ok = false; break; }
+        if (!wait(&ds_full[buf], (b >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         {
           const uint32_t k_lo = s0 + uint32_t((L::K_OFF + ((gk + j) % KST) * L::TILE) >> 4) + kMN;
@@ -279,7 +282,8 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const float nl2 = row_valid ? -p.lse[row_base + q_row] * kLog2e : 0.f;   // -lse, exp2 domain
       const float nd = row_valid ? -p.dvec[row_base + q_row] : 0.f;            // -D
       const uint64_t nl2x2 = f2_make(nl2, nl2), ndx2 = f2_make(nd, nd);
-      const uint64_t z_row = DROPOUT ? dropout_z(p.seed, (row_base + uint64_t(q_row)) * uint64_t(p.N)) : 0ull;
+      const uint64_t z_row = DROPOUT ? dropout_z(p.seed, (row_base + uint64_t(q_row)) * dropout_row_draws(p.N)) : 0ull;
+      const uint32_t drop_c = dropout_lane_c(p.drop_thr);
       for (int j = 0; j < n; ++j) {
         const int b = gb + j, buf = b & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(&s_full[buf], (b >> 1) & 1, wc))) { ok = false; break; }
@@ -311,7 +315,7 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (!__all_sync(0xffffffffu, mbar_wait(dp_full, b & 1, wc))) { ok = false; break; }
         tc_fence_after();
-        const uint64_t z_blk = z_row + uint64_t(k0) * kDropGamma;
+        const uint64_t z_blk = z_row + uint64_t(k0 >> 2) * kDropGamma;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {   // dS = P (dP Z/(1-p) - D), 64 keys at a time
           uint32_t dr[64];
@@ -326,14 +330,22 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (lane == 0) mbar_arrive(dp_read);
           }
           uint32_t pk[32];
+          uint32_t fl_hi = 0u;   // dropout: keep flags of keys 4u+2, 4u+3 (the draw's high word)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int c = 64 * hh + 2 * e;
             float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
             if (DROPOUT) {
-              const uint64_t z0 = z_blk + uint64_t(c) * kDropGamma;
-              dpa = dropout_bits_z(z0) >= p.drop_thr ? dpa * p.drop_scale : 0.f;
-              dpb = dropout_bits_z(z0 + kDropGamma) >= p.drop_thr ? dpb * p.drop_scale : 0.f;
+              uint32_t fl;
+              if ((e & 1) == 0) {   // one draw for keys c .. c+3
+                const uint64_t x = dropout_mix(z_blk + uint64_t(c >> 2) * kDropGamma);
+                fl = dropout_flags(uint32_t(x), drop_c);
+                fl_hi = dropout_flags(uint32_t(x >> 32), drop_c);
+              } else {
+                fl = fl_hi;
+              }
+              dpa = (fl & 0x8000u) ? dpa * p.drop_scale : 0.f;
+              dpb = (fl & 0x80000000u) ? dpb * p.drop_scale : 0.f;
             }
             float da, db;
             f2_split(f2_mul(f2_make(pr[c], pr[c + 1]), f2_add(f2_make(dpa, dpb), ndx2)), da, db);
@@ -345,7 +357,7 @@ fa_bwd_dq_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ds_full);
+        if (lane == 0) mbar_arrive(&ds_full[buf]);
       }
       if (!ok) break;
       // ---- epilogue: dq = bf16(tau * dQ)

@@ -143,8 +143,8 @@ struct BwdLayout {
   static constexpr int BAR_OFF = ITEM_OFF + NQI * 4;
   // kv_full, q_full[QS], q_empty[QS], stat_full[QS], do_full[DS], do_empty[DS], s_full, dp_full,
   // p_full[2], ds_full[2], dq_full, dq_empty, ds_free, fin, keep_full[2], kv_empty, dk_free,
-  // item_full[NQI], item_empty[NQI]
-  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 10 + 2 + 2 + 2 * NQI;
+  // item_full[NQI], item_empty[NQI], keep_empty[2]
+  static constexpr int NBARS = 1 + 3 * QS + 2 * DS + 10 + 2 + 2 + 2 * NQI + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   // TMEM: S^T, then (P*Z)^T over [0,64); dP^T, then dS^T over [128,192), then dQ^T; dV; dK
@@ -183,24 +183,56 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Keep bits of the 128 query columns of tile `qrow0` for key `key`: bit b of word w is the decision
-// for query qrow0 + 32 w + b.  Counters of consecutive queries are N apart.
-__device__ __forceinline__ uint4 keep_bits_row(const BwdParams& p, uint64_t row_base, int qrow0, int key) {
-  const uint64_t ctr0 = (row_base + uint64_t(qrow0)) * uint64_t(p.N) + uint64_t(key);
-  const uint64_t step = uint64_t(p.N) * kDropGamma;
-  uint64_t z = dropout_z(p.seed, ctr0);
-  uint32_t w[4];
+// Keep bits of the 128 query columns of tile `qrow0` for key k0 + r, made together by the four
+// lanes that hold keys k0 + 4m .. k0 + 4m + 3 (m = r >> 2; r & 3 = lane & 3): lane s = r & 3 takes
+// the draws of queries qrow0 + 4t + s (t = 0..31), each deciding the group's four keys, and a 4 x 4
+// exchange of 32-bit words gives every lane its own key's bits.  Every lane of the warp calls it.
+// Layout of the result: query column c of the tile, c = 64 qh + c', is bit
+// 16 (c' & 1) + (c' >> 2) of word 2 qh + ((c' >> 1) & 1); keep_bit() reads it.
+__device__ __forceinline__ uint4 keep_bits_row(const BwdParams& p, uint64_t row_base, int qrow0, int k0, int r) {
+  const uint32_t s = uint32_t(r) & 3u;
+  const uint64_t W = dropout_row_draws(p.N);
+  uint64_t z = dropout_z(p.seed, (row_base + uint64_t(qrow0) + s) * W + uint64_t((k0 >> 2) + (r >> 2)));
+  const uint64_t step = 4ull * W * kDropGamma;   // four queries on
+  const uint32_t c = dropout_lane_c(p.drop_thr);
+  // acc[hf]: keys 0 (bits 0-15) and 1 (bits 16-31) for t = 16 hf + bit; acc[2 + hf]: keys 2 and 3
+  uint32_t acc[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t bits = 0;
-#pragma unroll 8
-    for (int b = 0; b < 32; ++b) {
-      bits |= (dropout_bits_z(z) >= p.drop_thr ? 1u : 0u) << b;
+  for (int hf = 0; hf < 2; ++hf) {
+    uint32_t x01 = 0u, x23 = 0u;
+#pragma unroll 4
+    for (int tt = 0; tt < 16; ++tt) {
+      const uint64_t x = dropout_mix(z);
       z += step;
+      x01 |= ((dropout_flags(uint32_t(x), c) >> 15) & 0x00010001u) << tt;
+      x23 |= ((dropout_flags(uint32_t(x >> 32), c) >> 15) & 0x00010001u) << tt;
     }
-    w[i] = bits;
+    acc[hf] = x01;
+    acc[2 + hf] = x23;
   }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+  // v[kk]: key kk's bits for queries 4t + s, bit t
+  uint32_t v[4];
+  v[0] = __byte_perm(acc[0], acc[1], 0x5410);
+  v[1] = __byte_perm(acc[0], acc[1], 0x7632);
+  v[2] = __byte_perm(acc[2], acc[3], 0x5410);
+  v[3] = __byte_perm(acc[2], acc[3], 0x7632);
+  auto pick = [&](uint32_t i) { return (i & 2u) ? ((i & 1u) ? v[3] : v[2]) : ((i & 1u) ? v[1] : v[0]); };
+  // u[j] = lane j's word for this lane's key (queries 4t + j)
+  uint32_t rr[4];
+  rr[0] = pick(s);
+#pragma unroll
+  for (int d = 1; d < 4; ++d) rr[d] = __shfl_xor_sync(0xffffffffu, pick(s ^ uint32_t(d)), d);
+  auto from = [&](uint32_t j) {   // u[j] = rr[j ^ s]
+    const uint32_t i = j ^ s;
+    return (i & 2u) ? ((i & 1u) ? rr[3] : rr[2]) : ((i & 1u) ? rr[1] : rr[0]);
+  };
+  const uint32_t u0 = from(0), u1 = from(1), u2 = from(2), u3 = from(3);
+  return make_uint4(__byte_perm(u0, u1, 0x5410), __byte_perm(u2, u3, 0x5410), __byte_perm(u0, u1, 0x7632),
+                    __byte_perm(u2, u3, 0x7632));
+}
+// The keep bit of query column c' (0..63) of a half from that half's two words.
+__device__ __forceinline__ uint32_t keep_bit(const uint32_t (&kb)[2], int c) {
+  return (kb[(c >> 1) & 1] >> (16 * (c & 1) + (c >> 2))) & 1u;
 }
 
 // Register split per warpgroup (launch: 512 threads x 128 = 65536 registers):
@@ -324,6 +356,9 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* kv_empty = keep_full + 2; // per item: K and V may be replaced
   uint64_t* dk_free = kv_empty + 1;   // per item: the dK epilogue has read the accumulator
   const ItemQueue queue{reinterpret_cast<volatile int*>(smem + L::ITEM_OFF), dk_free + 1, dk_free + 1 + L::NQI, L::NQI};
+  // [2]: stage; the compute warps have read the keep bits of the stage's tile (used without DQ,
+  // where no dQ^T MMA orders the keep-bit warps behind the compute warps)
+  uint64_t* keep_empty = dk_free + 1 + 2 * L::NQI;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   float* stat = reinterpret_cast<float*>(smem + L::STAT_OFF);
@@ -349,6 +384,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_init(&p_full[h], 4);
       mbar_init(&ds_full[h], 4);
       mbar_init(&keep_full[h], 4);
+      mbar_init(&keep_empty[h], 8);
     }
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 4);
@@ -652,7 +688,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int qc0 = qrow0 + 64 * qh;         // first query of this half
       const float* st_l = stat + sq * 256 + 64 * qh;
       const bool need_mask = (k0 + 128 > kv_end) || (qc0 + 64 > p.N) || (p.causal && q_first + t == kt);
-      uint32_t kb[2] = {0u, 0u};   // dropout keep bits of this key row: query 64 qh + c -> bit c % 32 of kb[c / 32]
+      uint32_t kb[2] = {0u, 0u};   // dropout keep bits of this key row and query half (keep_bit)
       if (DROPOUT) {
         if (!warp_wait(&keep_full[g & 1], (g >> 1) & 1, wc)) { ok = false; break; }
         const uint2 w = reinterpret_cast<const uint2*>(&keep_smem[(g & 1) * 128 + r])[qh];
@@ -703,9 +739,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int e = 0; e < 32; ++e) {
           float a = pr[2 * e], bb = pr[2 * e + 1];
           if (DROPOUT) {   // P * Z; dV takes the 1/(1-p) factor in its fp32 epilogue
-            const uint32_t kbits = kb[e >> 4];
-            a = ((kbits >> ((2 * e) & 31)) & 1u) ? a : 0.f;
-            bb = ((kbits >> ((2 * e + 1) & 31)) & 1u) ? bb : 0.f;
+            a = keep_bit(kb, 2 * e) ? a : 0.f;
+            bb = keep_bit(kb, 2 * e + 1) ? bb : 0.f;
           }
           pk[e] = pack_bf16x2(a, bb);
         }
@@ -746,9 +781,8 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           const float4 nd = nd4[c >> 2];
           float dpa = __uint_as_float(dr[2 * e]), dpb = __uint_as_float(dr[2 * e + 1]);
           if (DROPOUT) {
-            const uint32_t kbits = kb[cc];
-            dpa = ((kbits >> (c & 31)) & 1u) ? dpa * p.drop_scale : 0.f;
-            dpb = ((kbits >> ((c + 1) & 31)) & 1u) ? dpb * p.drop_scale : 0.f;
+            dpa = keep_bit(kb, c) ? dpa * p.drop_scale : 0.f;
+            dpb = keep_bit(kb, c + 1) ? dpb * p.drop_scale : 0.f;
           }
           float da, db;   // dS = P (dP - D), as P * (dP + (-D)) on pairs
           const uint64_t nd2 = (e & 1) ? f2_make(nd.z, nd.w) : f2_make(nd.x, nd.y);
@@ -771,6 +805,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[qh]);
+      if (!DQ && DROPOUT && lane == 0) mbar_arrive(&keep_empty[g & 1]);   // its keep bits are read
     }
     if (!ok) break;
     // ---- dV epilogue: this half of the feature columns
@@ -816,7 +851,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       ok = ahead.start(p, queue, wc);
       for (int s2 = 0; ok && s2 < 2 && ahead.valid; ++s2) {   // the first two tiles
         keep_smem[s2 * 128 + r] =
-            keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0 + r);
+            keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0, r);
         __syncwarp();
         if (lane == 0) mbar_arrive(&keep_full[s2]);
         ok = ahead.advance(p, queue, wc);
@@ -832,16 +867,17 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int key = itm.k0 + r;
       for (int t = 0; t < itm.n_iter; ++t, ++g) {
         const int qrow0 = (itm.q_first + t) * 128;
-        if (!DQ) {   // only the keep bits: wait until the compute warps have finished tile g
-          if (DROPOUT) {
-            if (!warp_wait(&ds_full[0], g & 1, wc) || !warp_wait(&ds_full[1], g & 1, wc)) { ok = false; break; }
-            if (ahead.valid) {
-              keep_smem[(g & 1) * 128 + r] =
-                  keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0 + r);
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&keep_full[g & 1]);
-              if (!ahead.advance(p, queue, wc)) { ok = false; break; }
-            }
+        if (!DQ) {   // only the keep bits: wait until the compute warps have read those of tile g.
+          // (Not ds_full: the compute warps may complete two more tiles before this warp waits,
+          // and a parity wait cannot tell a barrier two phases on from one that has not moved.
+          // keep_empty of tile g + 2 needs the bits made here, so it cannot run ahead.)
+          if (DROPOUT && ahead.valid) {
+            if (!warp_wait(&keep_empty[g & 1], (g >> 1) & 1, wc)) { ok = false; break; }
+            keep_smem[(g & 1) * 128 + r] =
+                keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0, r);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&keep_full[g & 1]);
+            if (!ahead.advance(p, queue, wc)) { ok = false; break; }
           }
           continue;
         }
@@ -877,7 +913,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // free for the tile two ahead
         if (DROPOUT && ahead.valid) {
           keep_smem[(g & 1) * 128 + r] =
-              keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0 + r);
+              keep_bits_row(p, ahead.it.row_base, (ahead.it.q_first + ahead.t) * 128, ahead.it.k0, r);
           __syncwarp();
           if (lane == 0) mbar_arrive(&keep_full[g & 1]);
           if (!ahead.advance(p, queue, wc)) { ok = false; break; }

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -122,9 +123,10 @@ fa_status launch_status(const char* what) {
   return FA_OK;
 }
 
+// The 15-bit dropout threshold: a column is kept when its 15-bit draw is >= this value.
 uint32_t drop_threshold(float p) {
-  const double t = std::floor(double(p) * 4294967296.0);
-  return uint32_t(t > 4294967295.0 ? 4294967295.0 : t);
+  const double t = std::floor(double(p) * 32768.0);
+  return uint32_t(t > 32767.0 ? 32767.0 : t);
 }
 
 struct Workspace {
@@ -295,25 +297,56 @@ fa::BwdParams bwd_params(int B, int H, int N, float scale, int causal, const int
   return p;
 }
 
-// Key-range split of the decode kernel: about 296 CTAs in all (two per SM of a B200), at least
-// 512 keys per split, in whole 128-key blocks.  Host arithmetic only, so that the workspace size
-// needs no device.
+// Key-range split of the decode kernel.  Its shared memory holds one CTA per SM, so a grid of
+// BH * n CTAs runs in ceil(BH * n / sms) waves, each as long as one split's keys.  n minimises
+// waves * (chunk + 256): the 256 stands for a split's fixed cost (Q load, pipeline fill, partial
+// write) in keys.  Chunks are whole 128-key blocks of at least 512 keys; n <= 4 * sms.  With no SM
+// count (sms <= 0) the split is the finest one, n = ceil(Nkv / 512), which bounds the workspace of
+// every device.  Host arithmetic only.
 struct DecodeSplit {
   int chunk, n_split;
 };
-DecodeSplit decode_split(int BH, int Nkv) {
-  const long long want = (296 + BH - 1) / BH;                        // splits per head
-  long long chunk = (Nkv + want - 1) / want;
-  chunk = (chunk + 127) / 128 * 128;
-  if (chunk < 512) chunk = 512;
-  const long long n = (Nkv + chunk - 1) / chunk;
-  return DecodeSplit{int(chunk), int(n < 1 ? 1 : n)};
+DecodeSplit decode_split(int BH, int Nkv, int sms) {
+  auto chunk_for = [&](long long n) {
+    long long c = (Nkv + n - 1) / n;
+    c = (c + 127) / 128 * 128;
+    return c < 512 ? 512LL : c;
+  };
+  const long long finest = (Nkv + 511) / 512;
+  if (sms <= 0) {
+    const long long c = chunk_for(finest);
+    return DecodeSplit{int(c), int((Nkv + c - 1) / c)};
+  }
+  const long long top = std::min<long long>(finest, 4LL * sms);
+  DecodeSplit best{0, 0};
+  long long best_cost = -1;
+  for (long long n = 1; n <= top; ++n) {
+    const long long c = chunk_for(n);
+    const long long splits = (Nkv + c - 1) / c;
+    const long long waves = (BH * splits + sms - 1) / sms;
+    const long long cost = waves * (c + 256);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = DecodeSplit{int(c), int(splits)};
+    }
+  }
+  return best;
+}
+// SM count of the current device for the decode split, or 0 with no visible device (the CUDA error
+// that the query leaves is cleared, and the library's error message is left alone).
+int decode_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 size_t decode_o_bytes(int BH, int n_split, int Nq, int d) {
   return (size_t(BH) * n_split * Nq * d * 4 + 255) & ~size_t(255);
 }
-size_t decode_ws_bytes(int BH, int Nq, int Nkv, int d) {
-  const DecodeSplit sp = decode_split(BH, Nkv);
+size_t decode_ws_bytes(int BH, int Nq, int Nkv, int d, int sms) {
+  const DecodeSplit sp = decode_split(BH, Nkv, sms);
   return decode_o_bytes(BH, sp.n_split, Nq, d) + ((size_t(BH) * sp.n_split * Nq * 2 * 4 + 255) & ~size_t(255));
 }
 
@@ -620,7 +653,12 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 
 size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nkv, int d) {
   if (B < 1 || H < 1 || Nq < 1 || Nkv < 1 || d < 1) return 0;
-  return decode_ws_bytes(B * H, Nq, Nkv, d);
+  return decode_ws_bytes(B * H, Nq, Nkv, d, decode_sms());
+}
+
+int fa_fwd_decode_split(int B, int H, int Nkv, int sms) {
+  if (B < 1 || H < 1 || Nkv < 1) return 0;
+  return decode_split(B * H, Nkv, sms).n_split;
 }
 
 fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
@@ -637,9 +675,10 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   if (workspace == nullptr) return fail(FA_ERR_INVALID_ARG, "workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(FA_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
-  const size_t need = decode_ws_bytes(B * H, Nq, Nkv, d);
+  const int sms = decode_sms();
+  const size_t need = decode_ws_bytes(B * H, Nq, Nkv, d, sms);
   if (workspace_bytes < need) return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
-  const DecodeSplit sp = decode_split(B * H, Nkv);
+  const DecodeSplit sp = decode_split(B * H, Nkv, sms);
   CUtensorMap mq, mk, mv;
   if ((st = make_tile_map(&mq, q, B * H, Nq, d, "q", 64)) != FA_OK) return st;
   if ((st = make_tile_map(&mk, k, B * H, Nkv, d, "k")) != FA_OK) return st;
@@ -673,7 +712,7 @@ fa_status fa_dropout_mask(uint8_t* keep, int B, int H, int N, float dropout_p, u
   if (st != FA_OK) return st;
   const unsigned cap = unsigned(sms) * 32u;   // grid-stride loop: 32 blocks of 256 threads per SM
   const unsigned grid = grid_for(total, 256) > cap ? cap : grid_for(total, 256);
-  fa::fa_dropout_mask_kernel<<<grid, 256, 0, s>>>(keep, total, seed, drop_threshold(dropout_p));
+  fa::fa_dropout_mask_kernel<<<grid, 256, 0, s>>>(keep, total, N, seed, drop_threshold(dropout_p));
   return launch_status("fa_dropout_mask kernel launch");
 }
 

@@ -262,7 +262,8 @@ fa_fwd256_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const int q0 = qt * 128, q_row = q0 + r;
       const int kv_x = kv_end_of(qt, bh);
       const uint64_t z_row =
-          DROPOUT ? dropout_z(p.seed, (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * uint64_t(p.N)) : 0ull;
+          DROPOUT ? dropout_z(p.seed, (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * dropout_row_draws(p.N)) : 0ull;
+      const uint32_t drop_c = dropout_lane_c(p.drop_thr);
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const int b = gb + j, buf = b & 1;
@@ -313,8 +314,9 @@ fa_fwd256_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t negm2 = f2_make(-m_use, -m_use);
         uint64_t rs2 = f2_make(0.f, 0.f);
-        const uint64_t z_blk = z_row + uint64_t(k0) * kDropGamma;
+        const uint64_t z_blk = z_row + uint64_t(k0 >> 2) * kDropGamma;
         uint32_t pk[32];
+        uint32_t dm_hi = 0u;   // dropout: keep mask of keys 4u+2, 4u+3 (the draw's high word)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {   // pair e: keys 2e, 2e + 1 of the block
           const uint64_t x = f2_fma(f2_make(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2x2, negm2);
@@ -324,12 +326,16 @@ fa_fwd256_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           rs2 = f2_add(rs2, pp);
           float p0, p1;
           f2_split(pp, p0, p1);
-          if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
-            const uint64_t z0 = z_blk + uint64_t(2 * e) * kDropGamma;
-            p0 = dropout_bits_z(z0) >= p.drop_thr ? p0 : 0.f;
-            p1 = dropout_bits_z(z0 + kDropGamma) >= p.drop_thr ? p1 : 0.f;
-          }
           pk[e] = pack_bf16x2(p0, p1);
+          if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
+            if ((e & 1) == 0) {   // one draw for keys 2e .. 2e+3
+              const uint64_t xd = dropout_mix(z_blk + uint64_t(e >> 1) * kDropGamma);
+              dm_hi = dropout_mask2(dropout_flags(uint32_t(xd >> 32), drop_c));
+              pk[e] &= dropout_mask2(dropout_flags(uint32_t(xd), drop_c));
+            } else {
+              pk[e] &= dm_hi;
+            }
+          }
         }
         tmem_st32(lane_base + 64 * buf, pk);   // P over the block's score columns, already read
         tmem_st_wait();

@@ -17,9 +17,9 @@
 //              softmax runs, the tensor core works on the other tile.  P is handed over in two
 //              halves of 64 keys, so the first half of PV runs while the second half of P is made.
 // Softmax arithmetic: the scale-and-shift and the row sum use packed f32x2 operations and the row
-// max a tree of three-input maxima. At d=128 every exponential goes to the MUFU unit (moving a
-// share to a polynomial on the FMA pipe was measured slower there); at d=64 without dropout a
-// quarter of them take the FMA pipe (see kFmaPairsPer8).
+// max a tree of three-input maxima. Without dropout a quarter of the exponentials take a
+// polynomial on the FMA pipe and the rest the MUFU unit (see kFmaPairsPer8); with dropout all go to
+// the MUFU unit.
 // TMEM columns: S_A [0,128), S_B [128,256) (P over the first 64 columns of each), O_A [256,256+D),
 // O_B [256+D,256+2D).  tcgen05 operations from one thread complete in issue order, so S_X(j+1)
 // (which overwrites P_X(j)) runs after PV_X(j), and its completion also means PV_X(j) is done.
@@ -409,9 +409,10 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const int q_row = q0x + r;
       const int n = tile_n_kv(pair, bh, x);
       const int kv_x = tile_kv_end(pair, bh, x);
-      const uint64_t drop_row = (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * uint64_t(p.N);
-      // counter-hash state of key 0 of this row; key j adds j * gamma
-      const uint64_t z_row = DROPOUT ? dropout_z(p.seed, drop_row) : 0ull;
+      // counter-hash state of the draw of keys 0-3 of this row; keys 4u..4u+3 add u * gamma
+      const uint64_t z_row =
+          DROPOUT ? dropout_z(p.seed, (uint64_t(bh) * uint64_t(p.N) + uint64_t(q_row)) * dropout_row_draws(p.N)) : 0ull;
+      const uint32_t drop_c = dropout_lane_c(p.drop_thr);
       float m_ref = -INFINITY;   // reference max, exp2 domain
       float l = 0.f;
       for (int j = 0; j < n; ++j) {
@@ -449,10 +450,11 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t negm2 = f2_make(-m_use, -m_use);
         uint64_t rs2 = f2_make(0.f, 0.f);
-        const uint64_t z_blk = z_row + uint64_t(k0) * kDropGamma;
+        const uint64_t z_blk = z_row + uint64_t(k0 >> 2) * kDropGamma;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {   // two halves of 64 keys; the MMA takes each half as soon as it is ready
           uint32_t pk[32];
+          uint32_t dm_hi = 0u;   // dropout: keep mask of keys 4u+2, 4u+3 (the draw's high word)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int c = 32 * h + e;   // pair index: keys 2c, 2c+1
@@ -462,12 +464,16 @@ fa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             rs2 = kFmaPairsPer8<D, DROPOUT> > 0 ? f2_add_ftz(rs2, pp) : f2_add(rs2, pp);
             float p0, p1;
             f2_split(pp, p0, p1);
-            if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
-              const uint64_t z0 = z_blk + uint64_t(2 * c) * kDropGamma;
-              p0 = dropout_bits_z(z0) >= p.drop_thr ? p0 : 0.f;
-              p1 = dropout_bits_z(z0 + kDropGamma) >= p.drop_thr ? p1 : 0.f;
-            }
             pk[e] = pack_bf16x2(p0, p1);
+            if (DROPOUT) {   // Z only; the 1/(1-p) factor is applied in fp32 in the epilogue
+              if ((c & 1) == 0) {   // one draw for keys 2c .. 2c+3
+                const uint64_t x = dropout_mix(z_blk + uint64_t(c >> 1) * kDropGamma);
+                dm_hi = dropout_mask2(dropout_flags(uint32_t(x >> 32), drop_c));
+                pk[e] &= dropout_mask2(dropout_flags(uint32_t(x), drop_c));
+              } else {
+                pk[e] &= dm_hi;
+              }
+            }
           }
           // P over the score columns already read; O already holds PV up to block j-1
           tmem_st32(s_addr + 32 * h, pk);

@@ -84,8 +84,7 @@ __global__ void __launch_bounds__(128) fa_fwd_f32_kernel(const F32Params p) {
       float pr = expf(s - m);
       l += pr;
       if (p.dropout) {
-        const uint64_t ctr = (base + uint64_t(row)) * uint64_t(p.N) + uint64_t(j);
-        pr = dropout_keep(p.seed, ctr, p.drop_thr) ? pr * p.drop_scale : 0.f;
+        pr = dropout_keep(p.seed, base + uint64_t(row), dropout_row_draws(p.N), j, p.drop_thr) ? pr * p.drop_scale : 0.f;
       }
 #pragma unroll
       for (int c = 0; c < HALF; ++c) acc[c] = fmaf(pr, vs[jj][half * HALF + c], acc[c]);
@@ -102,10 +101,11 @@ __global__ void __launch_bounds__(128) fa_fwd_f32_kernel(const F32Params p) {
   }
 }
 
-__global__ void __launch_bounds__(256) fa_dropout_mask_kernel(uint8_t* keep, uint64_t total, uint64_t seed,
+__global__ void __launch_bounds__(256) fa_dropout_mask_kernel(uint8_t* keep, uint64_t total, int N, uint64_t seed,
                                                               uint32_t thr) {
+  const uint64_t W = dropout_row_draws(N);
   for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += uint64_t(gridDim.x) * blockDim.x)
-    keep[i] = dropout_keep(seed, i, thr) ? 1 : 0;
+    keep[i] = dropout_keep(seed, i / uint64_t(N), W, int(i % uint64_t(N)), thr) ? 1 : 0;
 }
 
 }  // namespace fa

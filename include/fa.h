@@ -152,11 +152,19 @@ FA_API size_t fa_bwd_noalloc_max_scratch(void);
  * Sequence b holds L = key_lens[b] valid keys (key_lens: int32 [B] on the device, or NULL for all
  * Nkv); query i is the token at position L - Nq + i, so causal keeps key j <= L - Nq + i and key
  * padding keeps j < L.  A query with no allowed key gets O = 0 and lse = -inf.  No dropout.
- * d in {64, 128}.  The key range of each head is split over CTAs that write fp32 partials
- * (m, l, unnormalised O) into the caller's workspace (at least fa_fwd_decode_workspace_size()
- * bytes, 256-byte aligned, clobbered; not shared by calls that may overlap), then a second launch
- * merges them.  Two kernel launches. */
+ * d in {64, 128}.  The key range of each head is split over CTAs (fa_fwd_decode_split splits
+ * per head) that write fp32 partials (m, l, unnormalised O) into the caller's workspace (at least
+ * fa_fwd_decode_workspace_size() bytes, 256-byte aligned, clobbered; not shared by calls that may
+ * overlap), then a second launch merges them.  Two kernel launches.
+ * The workspace size depends on the current device's SM count; with no visible device it is the
+ * size for the finest split (512-key chunks), enough on any device.  fa_fwd_decode returns
+ * FA_ERR_INVALID_ARG when the workspace is smaller than the current device needs. */
 FA_API size_t fa_fwd_decode_workspace_size(int B, int H, int Nq, int Nkv, int d);
+/* Number of key-range splits per head that fa_fwd_decode uses for B*H heads of Nkv keys on a device
+ * of `sms` SMs (sms <= 0: the finest split).  The split kernel holds one CTA per SM, so the choice
+ * minimises waves x (chunk + 256 keys of fixed cost per split) over chunks of whole 128-key blocks,
+ * at least 512 keys.  Host arithmetic only; 0 for B, H or Nkv < 1. */
+FA_API int fa_fwd_decode_split(int B, int H, int Nkv, int sms);
 FA_API fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int H, int Nq, int Nkv, int d, float scale, int causal,
                         const int32_t* key_lens, void* workspace, size_t workspace_bytes,

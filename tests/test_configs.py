@@ -51,6 +51,15 @@ def test_full_workload(name):
     print(f"{name}: O max-abs {o_err:.3e}, lse {l_err:.3e}, rel-L2 {errs}")
     for n, e in errs.items():
         assert e <= GRAD_REL_L2, (n, e)
+    # the backward with dQ in its own pass, at full size: many items per persistent CTA (this is where
+    # its keep-bit warps must not fall two tiles behind the compute warps)
+    sq, sk, sv = api.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, key_lens_device(x), w.dropout_p, w.seed,
+                                   separate_dq=True)
+    api.check()
+    assert torch.equal(sk, dk) and torch.equal(sv, dv)
+    e = rel_l2(to_f64(sq), ref[0])
+    print(f"{name}: separate dQ pass rel-L2 {e:.3e}")
+    assert e <= GRAD_REL_L2, e
 
 
 def test_long_context_64k():

@@ -67,3 +67,31 @@ def test_decode_host_validation():
     st = lib.fa_fwd_decode(fake, fake, fake, fake, fake, 1, 1, 4, 128, 64, 0.125, 0, None, 0x10000, need - 1, None)
     assert st == _lib.FA_ERR_INVALID_ARG and b"workspace" in lib.fa_get_error()
     assert lib.fa_fwd_decode_workspace_size(0, 1, 4, 128, 64) == 0
+
+
+def test_decode_split_fills_the_sms():
+    """The key-range split: one CTA per SM, so the grid should fill whole waves of SMs with as few
+    splits as that takes, in chunks of whole 128-key blocks of at least 512 keys."""
+    build()
+    lib = _lib.load()
+
+    def split(BH, Nkv, sms):
+        n = lib.fa_fwd_decode_split(1, BH, Nkv, sms)
+        chunk = -(-Nkv // n)
+        chunk = max(512, -(-chunk // 128) * 128)
+        assert -(-Nkv // chunk) == n   # every split holds keys
+        return n
+
+    assert split(16, 65536, 148) == 9            # 144 CTAs: one wave (19 splits took three)
+    assert split(16, 65536, 132) == 8            # 128 CTAs on a 132-SM part
+    assert split(1, 4096, 148) == 8              # one head: the finest split, 512 keys each
+    assert split(1, 1, 148) == 1
+    assert split(444, 4096, 148) == 1            # three full waves already
+    assert split(148, 65536, 148) == 1
+    assert split(16, 65536, 0) == 128            # no device: the finest split bounds the workspace
+    for BH, Nkv, sms in [(16, 65536, 148), (3, 5000, 148), (64, 32768, 148), (7, 100000, 148)]:
+        n = split(BH, Nkv, sms)
+        assert n <= split(BH, Nkv, 0)
+        waves = -(-BH * n // sms)
+        assert BH * n > (waves - 1) * sms       # no wave is empty
+    assert lib.fa_fwd_decode_split(0, 1, 10, 148) == 0

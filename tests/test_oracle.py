@@ -28,14 +28,15 @@ def _rand(shape, seed, factor=1.0):
 
 # ----------------------------------------------------------------------------- brute force
 def _bf_keep(seed, b, h, H, N, i, j, p):
-    """Pure-Python-int counter hash (pinned below to the published SplitMix64 stream)."""
-    ctr = ((b * H + h) * N + i) * N + j
-    z = (seed + (ctr + 1) * 0x9E3779B97F4A7C15) & M64
+    """Pure-Python-int counter hash (pinned below to the published SplitMix64 stream): one draw per
+    four key columns, a 15-bit field of its 16-bit lane j % 4 against floor(p 2^15)."""
+    g = ((b * H + h) * N + i) * ((N + 3) // 4) + j // 4
+    z = (seed + (g + 1) * 0x9E3779B97F4A7C15) & M64
     z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & M64
     z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & M64
     z ^= z >> 31
-    thr = min(math.floor(float(np.float32(p)) * 2.0 ** 32), 2 ** 32 - 1)
-    return (z >> 32) >= thr
+    thr = min(math.floor(float(np.float32(p)) * 2.0 ** 15), 2 ** 15 - 1)
+    return ((z >> (16 * (j % 4))) & 0x7FFF) >= thr
 
 
 def _brute_forward(q, k, v, scale, causal, key_lens, p, seed):
@@ -253,18 +254,26 @@ def test_hash_matches_published_splitmix64_stream():
         z = (int(ctr) + 1) * 0x9E3779B97F4A7C15 & M64   # seed 0
         got = int(splitmix64_mix(np.array([z], dtype=np.uint64))[0])
         assert got == int(want, 16)
-    # the per-element layout: (b, h, i, j) -> ctr = ((b*H + h)*N + i)*N + j
-    H, N = 3, 5
-    keep = keep_mask(0, 0, 0, H, N, [0], [0, 1, 2], 0.5)
-    expect = [(int(w, 16) >> 32) >= keep_threshold(0.5) for _, w in rows]
-    assert list(keep[0]) == expect
+    # the layout: (b, h, i, j) -> draw g = ((b*H + h)*N + i)*ceil(N/4) + j // 4, lane j % 4; with
+    # seed 0, row 0 of head 0 takes draws 0, 1, 2 for columns 0-3, 4-7, 8-11
+    H, N = 3, 13
+    for p in (0.5, 0.1, 0.9):
+        keep = keep_mask(0, 0, 0, H, N, [0], np.arange(12), p)
+        thr = math.floor(float(np.float32(p)) * 2 ** 15)
+        expect = [((int(w, 16) >> (16 * lane)) & 0x7FFF) >= thr for _, w in rows for lane in range(4)]
+        assert list(keep[0]) == expect
+    # a worked value: output 1 = 0xe220a8397b1dcdaf has 15-bit lanes 0x4daf, 0x7b1d, 0x2839, 0x6220
+    assert [((0xE220A8397B1DCDAF >> (16 * k)) & 0x7FFF) for k in range(4)] == [0x4DAF, 0x7B1D, 0x2839, 0x6220]
+    assert list(keep_mask(0, 0, 0, H, N, [0], [0, 1, 2, 3], 0.61)[0]) == [False, True, False, True]
+    # draws of the next row start at ceil(N/4) = 4: row 1, column 0 is output 5 of the stream
+    assert keep_mask(0, 0, 0, H, N, [1], [0], 0.5)[0, 0] == _bf_keep(0, 0, 0, H, N, 1, 0, 0.5)
 
 
 def test_threshold_and_rates():
     assert keep_threshold(0.0) == 0
-    assert keep_threshold(0.5) == 2 ** 31
-    assert keep_threshold(0.1) == math.floor(float(np.float32(0.1)) * 2 ** 32)
-    assert keep_threshold(0.9999999) <= 2 ** 32 - 1
+    assert keep_threshold(0.5) == 2 ** 14
+    assert keep_threshold(0.1) == 3276            # floor(0.1 * 32768): drop rate 0.09998
+    assert keep_threshold(0.9999999) == 2 ** 15 - 1
     w = WORKLOADS["bf16_keypad_dropout_16x16x512x64"]
     p, n, kept = w.dropout_p, 0, 0
     for b in range(w.B):
