@@ -29,11 +29,13 @@
 //   warp 12    producer: takes the work items (item queue below), TMA K and V per item, Q (2 deep)
 //              and dO (1 deep at D=128, 2 at D=64) per query tile
 //   warp 13    MMA issuer; warp 14 loads -lse and -D per query tile into shared memory; warp 15 idle
-// TMEM (512 columns): S^T [0,128), then (P*Z)^T; dP^T [128,256), then dS^T, then dQ^T;
-// dV [256,256+D); dK [256+D,256+2D).  MMA order per query tile t:
+// TMEM (512 columns): S^T [0,128), then (P*Z)^T; dP^T [128,256), then dS^T, then (D = 128) dQ^T;
+// dV [256,256+D); dK [256+D,256+2D); at D = 64 dQ^T has columns of its own, [384,512).  MMA order per
+// query tile t:
 //   dV_t (per query half), S_{t+1}, dK_t (per query half), dQ^T_t, dP_{t+1}
 // so S_{t+1} runs while the compute warps make dS_t, and dK_t reads dS^T before dQ^T_t overwrites it
-// (MMAs of one thread execute in issue order).
+// (MMAs of one thread execute in issue order).  At D = 128, dP_{t+1} waits until the dQ warps have
+// read dQ^T_t out of the shared columns; at D = 64 only dQ^T_{t+1} waits for that.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -149,6 +151,11 @@ struct BwdLayout {
   static constexpr int BYTES = MISC_OFF + 16;
   // TMEM: S^T, then (P*Z)^T over [0,64); dP^T, then dS^T over [128,192), then dQ^T; dV; dK
   static constexpr int ST_COL = 0, DPT_COL = 128, DV_COL = 256, DK_COL = 256 + D;
+  // dQ^T: at D = 64 in columns of its own [384, 512), so that dP_{t+1} need not wait until the dQ
+  // warps have read dQ^T_t out of the dP^T columns (only dQ^T_{t+1} waits for that); at D = 128 the
+  // 512 columns are taken and dQ^T goes over dP^T/dS^T
+  static constexpr int DQT_COL = (D == 64) ? 256 + 2 * D : DPT_COL;
+  static constexpr bool DQT_OWN = DQT_COL != DPT_COL;
   static constexpr int TMEM_COLS = 512;
   static_assert(DK_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
@@ -583,7 +590,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       if (!wait(&q_full[g % QS], (g / QS) & 1)) { ok = false; break; }
       tc_fence_after();
       issue_s(g);
-      if (DQ && g >= 1 && !wait(dq_empty, (g - 1) & 1)) { ok = false; break; }
+      if (DQ && !L::DQT_OWN && g >= 1 && !wait(dq_empty, (g - 1) & 1)) { ok = false; break; }
       if (!wait(&do_full[g % DS], (g / DS) & 1)) { ok = false; break; }
       tc_fence_after();
       issue_dp(g);
@@ -633,12 +640,14 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         mma_commit_elect(&q_empty[g % QS]);    // Q_g: last read by dK_g
         if (DQ) {
-          // dQ^T = K^T dS^T over the dS^T/dP^T columns, after dK_g has read them
-          // (M = D, N = 128 queries, K = 128 keys; B = dS^T from shared memory)
+          // dQ^T = K^T dS^T (M = D, N = 128 queries, K = 128 keys; B = dS^T from shared memory):
+          // over the dS^T/dP^T columns after dK_g has read them, or in its own columns once the dQ
+          // warps have read the previous tile's
+          if (L::DQT_OWN && g >= 1 && !wait(dq_empty, (g - 1) & 1)) { ok = false; break; }
           const uint32_t k_lo = lo(L::K_OFF, kMN), ds_lo = lo(L::DS_OFF, kMN);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss_elect(tmem + L::DPT_COL, sdesc_join(k_lo + kk * (2048 >> 4), kHi),
+            mma_ss_elect(tmem + L::DQT_COL, sdesc_join(k_lo + kk * (2048 >> 4), kHi),
                         sdesc_join(ds_lo + kk * (2048 >> 4), kHi), kIdQ, kk > 0 ? 1u : 0u);
           mma_commit_elect(dq_full);
           mma_commit_elect(ds_free);             // the shared-memory dS tile is free again
@@ -646,7 +655,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // dP_{g+1} once the dQ warps have read dQ^T out of those columns (with DQ; without it, the
         // dK MMAs issued above read dS^T there first: MMAs run in issue order)
         if (more) {
-          if (DQ && !wait(dq_empty, g & 1)) { ok = false; break; }
+          if (DQ && !L::DQT_OWN && !wait(dq_empty, g & 1)) { ok = false; break; }
           if (!wait(&do_full[(g + 1) % DS], ((g + 1) / DS) & 1)) { ok = false; break; }
           tc_fence_after();
           issue_dp(g + 1);
@@ -886,7 +895,7 @@ fa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint32_t gq[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          tmem_ld32(lane_base + L::DPT_COL + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&gq[32 * c]));
+          tmem_ld32(lane_base + L::DQT_COL + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&gq[32 * c]));
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&gq[h * 32]));
