@@ -138,8 +138,8 @@ TC_FLOP_PER_CLK_SM = 8192
 DATASHEET_BF16_TFLOPS = 2250.0
 
 
-def clock_peak_tflops(sm_mhz, sms=148):
-    """Tensor-core peak at the sampled SM clock: 8192 FLOP per clock per SM."""
+def clock_peak_tflops(sm_mhz, sms):
+    """Tensor-core peak at the sampled SM clock: 8192 FLOP per clock per SM, `sms` SMs."""
     return TC_FLOP_PER_CLK_SM * sms * sm_mhz * 1e6 / 1e12
 
 
@@ -161,6 +161,7 @@ def run_native(args, w, world, rank, local):
 
     x = make_inputs(w, exact=False)
     B, H, N, d = w.B, w.H, w.N, w.d
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     def up(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -320,12 +321,12 @@ def run_native(args, w, world, rank, local):
         "frac_of_datasheet": {"fwd": round(fwd_tflops / world / DATASHEET_BF16_TFLOPS, 4),
                               "fwd_bwd": round(tflops / world / DATASHEET_BF16_TFLOPS, 4)},
         "frac_of_clock_peak": None if mhz is None else {
-            "fwd": round(fwd_tflops / world / clock_peak_tflops(mhz), 4),
-            "fwd_bwd": round(tflops / world / clock_peak_tflops(mhz), 4),
-            "peak_tflops": round(clock_peak_tflops(mhz), 1), "sm_mhz": mhz},
+            "fwd": round(fwd_tflops / world / clock_peak_tflops(mhz, sms), 4),
+            "fwd_bwd": round(tflops / world / clock_peak_tflops(mhz, sms), 4),
+            "peak_tflops": round(clock_peak_tflops(mhz, sms), 1), "sm_mhz": mhz, "sms": sms},
         "peak_source": (f"targets use the {pk['source']} bf16 peak {pk['bf16_tflops']} TFLOP/s (cuBLAS burst); "
                         f"HBM {pk['hbm_gbs']} GB/s {pk['source']}; frac_of_datasheet divides by NVIDIA's dense bf16 "
-                        f"{DATASHEET_BF16_TFLOPS} TFLOP/s (HGX B200); frac_of_clock_peak by 8192 FLOP/clk/SM x 148 SMs "
+                        f"{DATASHEET_BF16_TFLOPS} TFLOP/s (HGX B200); frac_of_clock_peak by 8192 FLOP/clk/SM x {sms} SMs "
                         "at the median sampled SM clock"),
         "roofline": {"kernel": dom, "bound": "tensor", "achieved": round(dom_ach, 1), "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": round(dom_ach / pk["bf16_tflops"], 4),
@@ -337,6 +338,13 @@ def run_native(args, w, world, rank, local):
         "gpu_launches": 4 * args.steps,   # fused: fwd, prep, main, convert; split: fwd, prep, main, dQ pass
         "clocks": clocks,
     }
+    if x["key_lens"] is not None and not w.causal:
+        # key padding: every query row sees len_b keys, so the work done is sum_b len_b * N per head
+        # instead of the nominal N^2 (the metric's value stays the nominal count)
+        eff = float(np.sum(x["key_lens"].astype(np.float64))) / (B * N)
+        line["effective"] = {"fraction_of_nominal_flops": round(eff, 4),
+                             "fwd_bwd_tflops": round(tflops * eff, 2), "fwd_tflops": round(fwd_tflops * eff, 2),
+                             "note": "FLOPs counted over the allowed keys only: 4 d H N sum_b len_b forward"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
     return line
