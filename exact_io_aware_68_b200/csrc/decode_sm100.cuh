@@ -132,6 +132,9 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl wc{p.wait_ns, abort_flag};
+  // the combine kernel (a programmatic dependent launch) may be scheduled from here on; it waits
+  // for this whole grid before it reads anything
+  asm volatile("griddepcontrol.launch_dependents;");
 
   if (warp == 4) {
     // =========================================================== producer
@@ -353,6 +356,8 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 // Merge of the partials of one (head, query row) per warp: lanes take D/32 features each.
 template <int D>
 __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecodeParams p) {
+  // launched as a programmatic dependent of the split kernel: wait for that grid to complete
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int w = int(blockIdx.x) * 8 + (int(threadIdx.x) >> 5), lane = int(threadIdx.x) & 31;
   const int rows = p.B * p.H * p.Nq;
   if (w >= rows) return;

@@ -358,8 +358,22 @@ fa_status launch_decode(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   if (st != FA_OK) return st;
   fa::fa_decode_split_kernel<D><<<dim3(p.n_split, p.B * p.H), 192, L::BYTES, s>>>(mq, mk, mv, p);
   if ((st = launch_status("fa_fwd_decode split kernel launch")) != FA_OK) return st;
+  // The combine is a programmatic dependent launch: it may be scheduled while the split kernel
+  // runs and waits (griddepcontrol.wait) until that grid has completed and its writes are visible,
+  // so the second launch adds no gap of its own.
   const unsigned rows = unsigned(p.B * p.H * p.Nq);
-  fa::fa_decode_combine_kernel<D><<<(rows + 7) / 8, 256, 0, s>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((rows + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D>, p);
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "fa_fwd_decode combine kernel launch: %s", cudaGetErrorString(e));
   return launch_status("fa_fwd_decode combine kernel launch");
 }
 
