@@ -10,12 +10,16 @@
 // O = sum w_s O_s / sum w_s l_s, lse = (m* + log2 sum w_s l_s) ln 2.  Bound: HBM (every K and V byte
 // is read once; a row of Nq queries does Nq * 4 d FLOP per key).
 //
-// Split kernel, 6 warps:
-//   warps 0-3  softmax: the M = 64 query tile sits in TMEM lanes 32w .. 32w + 15 (row 16w + lane);
-//              one thread per query row, 128 keys per block; P (bf16) goes to shared memory
-//   warp 4     producer: Q once (64 rows, zero past Nq), K and V blocks of 128 keys through rings
-//   warp 5     MMA issuer: S(j) = Q K_j^T (M = 64, N = 128) into one of two TMEM score buffers, so
-//              that S(j+1) runs while block j is exponentiated; O += P(j) V_j (M = 64, N = D)
+// Split kernel, 6 warps, an M = 128 tile whose rows r and r + 64 hold the same query row r % 64:
+//   warps 0-3  softmax: thread r (TMEM lane r) exponentiates the key half r / 64 of every 128-key
+//              block (64 keys) for query row r % 64 and keeps its own running max and sum, so each
+//              half of a split's keys is a partial of its own for the combine (2 per CTA); P (bf16:
+//              its 64 keys, zeros for the other half) goes over the first 64 columns of the score
+//              buffer.  Half the exponentials per thread and block of a one-thread-per-row tile.
+//   warp 4     producer: Q twice (tile rows 0-63 and 64-127, zero past Nq), K and V rings
+//   warp 5     MMA issuer: S(j) = Q K_j^T (M = 128, N = 128) into one of two TMEM score buffers, so
+//              that S(j+1) runs while block j is exponentiated; O += P(j) V_j (M = 128, N = D, P from
+//              TMEM)
 // TMEM: S0 [0,128), S1 [128,256), O [256, 256+D).
 #pragma once
 #include <cuda_bf16.h>
@@ -27,14 +31,15 @@ constexpr float kDecodeRescale = 8.0f;   // move the reference max only when a b
 constexpr float kDecodeLn2 = 0.69314718055994530942f;
 
 struct DecodeParams {
-  float* part_o;               // [BH][n_split][Nq][D] fp32, unnormalised
-  float* part_ml;              // [BH][n_split][Nq][2] fp32: m (log2 domain), l
+  float* part_o;               // [BH][n_part][Nq][D] fp32, unnormalised
+  float* part_ml;              // [BH][n_part][Nq][2] fp32: m (log2 domain), l
   __nv_bfloat16* o;            // [B,H,Nq,D]
   float* lse;                  // [B,H,Nq]
   const int32_t* key_lens;     // [B] or null
   int B, H, Nq, Nkv;
   int chunk;                   // keys per split (multiple of 128)
-  int n_split;
+  int n_split;                 // key-range splits per head (CTAs per head)
+  int n_part;                  // partials per head: 2 per split (one per key half)
   int causal;
   float scale_log2;
   uint64_t wait_ns;
@@ -42,25 +47,23 @@ struct DecodeParams {
 
 template <int D>
 struct DecodeLayout {
-  static constexpr int QSUB = 64 * 128;          // one 64-column panel of the 64-row Q tile
-  static constexpr int KSUB = 128 * 128;         // one 64-column panel of a 128-row K/V block
-  static constexpr int QTILE = D / 64 * QSUB;
-  static constexpr int BLK = 128 * D * 2;
-  static constexpr int KST = (D == 128) ? 2 : 4;
+  static constexpr int SUB = 128 * 128;          // one 64-column (128-byte) panel of a 128-row tile
+  static constexpr int QHALF = 64 * 128;         // rows 64-127 of a panel start here
+  static constexpr int TILE = D / 64 * SUB;      // a 128-row bf16 tile (Q, or a K/V block)
+  static constexpr int KST = (D == 128) ? 3 : 4;
   static constexpr int VST = (D == 128) ? 2 : 4;
-  static constexpr int PBUF = 64 * 128 * 2;      // P of one block: 64 rows x 128 keys bf16 (2 panels)
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + QTILE;
-  static constexpr int V_OFF = K_OFF + KST * BLK;
-  static constexpr int P_OFF = V_OFF + VST * BLK;
-  static constexpr int BAR_OFF = P_OFF + 2 * PBUF;
+  static constexpr int K_OFF = Q_OFF + TILE;
+  static constexpr int V_OFF = K_OFF + KST * TILE;
+  static constexpr int BAR_OFF = V_OFF + VST * TILE;
   // q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2], s_free[2], p_full[2],
-  // p_free[2], pv_done, fin
-  static constexpr int NBARS = 1 + 2 * KST + 2 * VST + 8 + 2;
+  // pv_done, fin
+  static constexpr int NBARS = 1 + 2 * KST + 2 * VST + 6 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int O_COL = 256;
   static constexpr int TMEM_COLS = 512;
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
   static_assert(BYTES <= 232448, "shared memory budget");
 };
 
@@ -83,10 +86,9 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + VST;
   uint64_t* s_full = v_empty + VST;   // [2]
-  uint64_t* s_free = s_full + 2;      // [2]
-  uint64_t* p_full = s_free + 2;      // [2]
-  uint64_t* p_free = p_full + 2;      // [2]
-  uint64_t* pv_done = p_free + 2;     // one phase per block
+  uint64_t* s_free = s_full + 2;      // [2]: the softmax has read the scores out of the buffer
+  uint64_t* p_full = s_free + 2;      // [2]: P is in the buffer
+  uint64_t* pv_done = p_full + 2;     // one phase per block
   uint64_t* fin = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
@@ -95,8 +97,7 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   const int b = bh / p.H;
   int kv_len = p.Nkv;
   if (p.key_lens != nullptr) kv_len = min(kv_len, max(p.key_lens[b], 0));
-  // keys of this split that any query may see: below the cache length, and (causal) at most the
-  // position of the last query, L - 1
+  // the keys of this split below the cache length
   const int c0 = split * p.chunk;
   const int c1 = min(c0 + p.chunk, kv_len);
   const int n_blk = c1 > c0 ? (c1 - c0 + 127) / 128 : 0;
@@ -115,7 +116,6 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 4);
       mbar_init(&p_full[s], 4);
-      mbar_init(&p_free[s], 1);
     }
     mbar_init(pv_done, 1);
     mbar_init(fin, 1);
@@ -142,25 +142,30 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(q_full, L::QTILE);
+      // Q into tile rows 0-63 and again into rows 64-127 (the 128-byte swizzle repeats every 8 rows,
+      // so the second copy sits at the same phase)
+      mbar_arrive_expect_tx(q_full, L::TILE);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) tma_load_3d(smem + L::Q_OFF + c * L::QSUB, &tm_q, q_full, c * 64, 0, bh);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(smem + L::Q_OFF + c * L::SUB, &tm_q, q_full, c * 64, 0, bh);
+        tma_load_3d(smem + L::Q_OFF + c * L::SUB + L::QHALF, &tm_q, q_full, c * 64, 0, bh);
+      }
       int gk = 0, gv = 0;
       bool ok = true;
       for (int j = 0; ok && j < n_blk; ++j) {
         const int key0 = c0 + j * 128;
         // K_j, then V_j (V is needed one block later than K)
         if (gk >= KST && !mbar_wait(&k_empty[gk % KST], ((gk / KST) - 1) & 1, wc)) { ok = false; break; }
-        mbar_arrive_expect_tx(&k_full[gk % KST], L::BLK);
+        mbar_arrive_expect_tx(&k_full[gk % KST], L::TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::K_OFF + (gk % KST) * L::BLK + c * L::KSUB, &tm_k, &k_full[gk % KST], c * 64, key0, bh);
+          tma_load_3d(smem + L::K_OFF + (gk % KST) * L::TILE + c * L::SUB, &tm_k, &k_full[gk % KST], c * 64, key0, bh);
         ++gk;
         if (gv >= VST && !mbar_wait(&v_empty[gv % VST], ((gv / VST) - 1) & 1, wc)) { ok = false; break; }
-        mbar_arrive_expect_tx(&v_full[gv % VST], L::BLK);
+        mbar_arrive_expect_tx(&v_full[gv % VST], L::TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::V_OFF + (gv % VST) * L::BLK + c * L::KSUB, &tm_v, &v_full[gv % VST], c * 64, key0, bh);
+          tma_load_3d(smem + L::V_OFF + (gv % VST) * L::TILE + c * L::SUB, &tm_v, &v_full[gv % VST], c * 64, key0, bh);
         ++gv;
       }
       // every copy started here lands before the CTA releases its shared memory
@@ -172,41 +177,37 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   } else if (warp == 5) {
     // =========================================================== MMA issuer (whole warp, elect.sync)
     if (n_blk > 0) {
-      constexpr uint32_t kIdS = idesc_bf16(64, 128, false, false);   // Q: K-major, K: K-major
-      constexpr uint32_t kIdPV = idesc_bf16(64, D, false, true);     // P: K-major (smem), V: MN-major
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // Q: K-major, K: K-major
+      constexpr uint32_t kIdPV = idesc_bf16(128, D, false, true);     // P: TMEM, V: MN-major
       const uint32_t s0 = smem_u32(smem) >> 4;
-      constexpr uint32_t kHi = sdesc_sw128_hi(1024), kKM = sdesc_lbo(16), kMN = sdesc_lbo(L::KSUB);
+      constexpr uint32_t kHi = sdesc_sw128_hi(1024), kKM = sdesc_lbo(16), kMN = sdesc_lbo(L::SUB);
       auto wait = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc)); };
       auto issue_s = [&](int j) {   // S(j) = Q K_j^T into score buffer j % 2
         const uint32_t q_lo = s0 + uint32_t(L::Q_OFF >> 4) + kKM;
-        const uint32_t k_lo = s0 + uint32_t((L::K_OFF + (j % KST) * L::BLK) >> 4) + kKM;
+        const uint32_t k_lo = s0 + uint32_t((L::K_OFF + (j % KST) * L::TILE) >> 4) + kKM;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qo = ((kk >> 2) * L::QSUB + (kk & 3) * 32) >> 4;
-          const uint32_t ko = ((kk >> 2) * L::KSUB + (kk & 3) * 32) >> 4;
-          mma_ss_elect(tmem + 128 * (j & 1), sdesc_join(q_lo + qo, kHi), sdesc_join(k_lo + ko, kHi), kIdS,
+        for (int kk = 0; kk < D / 16; ++kk) {   // 16 features per step: 32 bytes inside a 128-byte row
+          const uint32_t off = ((kk >> 2) * L::SUB + (kk & 3) * 32) >> 4;
+          mma_ss_elect(tmem + 128 * (j & 1), sdesc_join(q_lo + off, kHi), sdesc_join(k_lo + off, kHi), kIdS,
                       kk > 0 ? 1u : 0u);
         }
         mma_commit_elect(&s_full[j & 1]);
         mma_commit_elect(&k_empty[j % KST]);
       };
-      auto issue_pv = [&](int j) {   // O += P(j) V_j   (A = P in shared memory, 64 rows x 128 keys)
-        const uint32_t p_lo = s0 + uint32_t((L::P_OFF + (j & 1) * L::PBUF) >> 4) + kKM;
-        const uint32_t v_lo = s0 + uint32_t((L::V_OFF + (j % VST) * L::BLK) >> 4) + kMN;
+      auto issue_pv = [&](int j) {   // O += P(j) V_j   (A = P over the first 64 columns of buffer j % 2)
+        const uint32_t v_lo = s0 + uint32_t((L::V_OFF + (j % VST) * L::TILE) >> 4) + kMN;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step
-          const uint32_t po = ((kk >> 2) * L::QSUB + (kk & 3) * 32) >> 4;
-          mma_ss_elect(tmem + L::O_COL, sdesc_join(p_lo + po, kHi), sdesc_join(v_lo + kk * (2048 >> 4), kHi), kIdPV,
-                      (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: 8 packed TMEM columns, 16 rows of V
+          mma_ts_elect(tmem + L::O_COL, tmem + 128 * (j & 1) + kk * 8, sdesc_join(v_lo + kk * (2048 >> 4), kHi),
+                      kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit_elect(&v_empty[j % VST]);
-        mma_commit_elect(&p_free[j & 1]);
         mma_commit_elect(pv_done);
       };
       bool ok = wait(q_full, 0);
       for (int j = 0; ok && j <= n_blk; ++j) {
         if (j < n_blk) {
-          // score buffer j % 2 was last read by the softmax of block j - 2
+          // buffer j % 2 held S(j-2), read by the softmax, and P(j-2), read by PV(j-2): issued in
+          // the previous iteration, so it runs first
           if (j >= 2 && !wait(&s_free[j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
           if (!wait(&k_full[j % KST], (j / KST) & 1)) { ok = false; break; }
           tc_fence_after();
@@ -226,41 +227,42 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     __syncwarp();
   } else {
     // =========================================================== softmax (warps 0-3)
-    // M = 64 layout: lanes 0..15 of warp w hold rows 16 w + lane; lanes 16..31 hold no row but join
-    // every warp-wide TMEM access.
-    const int row = 16 * warp + (lane & 15);
-    const bool has_row = lane < 16;
+    const int r = 32 * warp + lane;       // TMEM lane
+    const int half = r >> 6;              // keys [64 half, 64 half + 64) of every block
+    const int row = r & 63;               // query row
     const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_make(sl2, sl2);
     // position of this query in the cache, and the keys it may see
     const int pos = kv_len - p.Nq + row;
-    const int lim = (has_row && row < p.Nq) ? (p.causal ? min(kv_len, pos + 1) : kv_len) : 0;   // keys < lim allowed
+    const int lim = row < p.Nq ? (p.causal ? min(kv_len, pos + 1) : kv_len) : 0;   // keys < lim allowed
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* p_smem = smem + L::P_OFF;
+    uint32_t zero[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) zero[e] = 0u;
     for (int j = 0; j < n_blk; ++j) {
+      const uint32_t sbuf = lane_base + 128 * (j & 1);
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, wc))) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(lane_base + 128 * (j & 1) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+      uint32_t sr[64];
+      tmem_ld32(sbuf + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(sbuf + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
-#pragma unroll
-      for (int h = 0; h < 4; ++h) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32 * h]));
+      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[j & 1]);   // the MMA may overwrite this score buffer
-      const int k0 = c0 + 128 * j;
-      if (k0 + 128 > lim) {   // mask keys >= lim
+      if (lane == 0) mbar_arrive(&s_free[j & 1]);   // scores read: S(j+2) may follow PV(j)
+      const int k0 = c0 + 128 * j + 64 * half;
+      if (k0 + 64 > lim) {   // mask keys >= lim
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (k0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) mx = max3f(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+      for (int c = 0; c < 64; c += 2) mx = max3f(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
       const float m_cand = mx * sl2;
       float alpha = 1.f;
       if (m_cand > m_ref + kDecodeRescale) {
@@ -285,30 +287,24 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       const uint64_t negm2 = f2_make(-m_use, -m_use);
-      // the P buffer of block j - 2 has been read by its PV
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&p_free[j & 1], ((j - 2) >> 1) & 1, wc))) { ok = false; break; }
       uint64_t rs2 = f2_make(0.f, 0.f);
-      uint8_t* prow = p_smem + (j & 1) * L::PBUF + row * 128;
+      uint32_t pk[32];
 #pragma unroll
-      for (int chunk = 0; chunk < 16; ++chunk) {   // 8 keys per 16-byte chunk; panel = chunk / 8
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 8 * chunk + 2 * e;
-          const uint64_t x = f2_fma(f2_make(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm2);
-          float x0, x1;
-          f2_split(x, x0, x1);
-          const uint64_t pp = f2_make(ex2_approx(x0), ex2_approx(x1));
-          rs2 = f2_add(rs2, pp);
-          float p0, p1;
-          f2_split(pp, p0, p1);
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        if (has_row)
-          *reinterpret_cast<uint4*>(prow + (chunk >> 3) * L::QSUB + (((chunk & 7) ^ (row & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int e = 0; e < 32; ++e) {
+        const uint64_t x = f2_fma(f2_make(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2x2, negm2);
+        float x0, x1;
+        f2_split(x, x0, x1);
+        const uint64_t pp = f2_make(ex2_approx(x0), ex2_approx(x1));
+        rs2 = f2_add(rs2, pp);
+        float p0, p1;
+        f2_split(pp, p0, p1);
+        pk[e] = pack_bf16x2(p0, p1);
       }
-      fence_proxy_async_smem();   // generic-proxy stores -> visible to the tensor core
+      // P over the first 64 columns of the buffer (scores already read): this half's 64 keys and
+      // zeros for the other half (its query's other row holds those)
+      tmem_st32(sbuf + 32 * half, pk);
+      tmem_st32(sbuf + 32 * (1 - half), zero);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[j & 1]);
@@ -316,8 +312,8 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       f2_split(rs2, rs0, rs1);
       l = l * alpha + (rs0 + rs1);
     }
-    // ---- partial: unnormalised O, m (log2 domain), l
-    const uint64_t part = (uint64_t(bh) * p.n_split + split) * p.Nq + row;
+    // ---- partial of this key half: unnormalised O, m (log2 domain), l
+    const uint64_t part = (uint64_t(bh) * p.n_part + 2 * split + half) * p.Nq + row;
     if (n_blk > 0 && ok && __all_sync(0xffffffffu, mbar_wait(fin, 0, wc))) {
       tc_fence_after();
 #pragma unroll
@@ -326,7 +322,7 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tmem_ld32(lane_base + L::O_COL + 32 * c, orr);
         tmem_ld_wait();
         reg_fence32(orr);
-        if (has_row && row < p.Nq) {
+        if (row < p.Nq) {
           float4* dst = reinterpret_cast<float4*>(p.part_o + part * D + 32 * c);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
@@ -334,12 +330,12 @@ fa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                                  __uint_as_float(orr[4 * e + 2]), __uint_as_float(orr[4 * e + 3]));
         }
       }
-    } else if (n_blk == 0 && has_row && row < p.Nq) {
+    } else if (n_blk == 0 && row < p.Nq) {
       float4* dst = reinterpret_cast<float4*>(p.part_o + part * D);
 #pragma unroll
       for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (has_row && row < p.Nq) {
+    if (row < p.Nq) {
       p.part_ml[2 * part] = (l > 0.f) ? m_ref : -INFINITY;
       p.part_ml[2 * part + 1] = l;
     }
@@ -363,8 +359,8 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecodePara
   if (w >= rows) return;
   const int bh = w / p.Nq, i = w % p.Nq;
   float m_star = -INFINITY;
-  for (int s = lane; s < p.n_split; s += 32)
-    m_star = fmaxf(m_star, p.part_ml[2 * ((uint64_t(bh) * p.n_split + s) * p.Nq + i)]);
+  for (int s = lane; s < p.n_part; s += 32)
+    m_star = fmaxf(m_star, p.part_ml[2 * ((uint64_t(bh) * p.n_part + s) * p.Nq + i)]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m_star = fmaxf(m_star, __shfl_xor_sync(0xffffffffu, m_star, off));
   constexpr int PER = D / 32;
@@ -373,8 +369,8 @@ __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecodePara
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float l_star = 0.f;
   if (m_star != -INFINITY) {
-    for (int s = 0; s < p.n_split; ++s) {
-      const uint64_t part = (uint64_t(bh) * p.n_split + s) * p.Nq + i;
+    for (int s = 0; s < p.n_part; ++s) {
+      const uint64_t part = (uint64_t(bh) * p.n_part + s) * p.Nq + i;
       const float ms = p.part_ml[2 * part];
       if (ms == -INFINITY) continue;
       const float ws = ex2_approx(ms - m_star);

@@ -345,9 +345,11 @@ int decode_sms() {
 size_t decode_o_bytes(int BH, int n_split, int Nq, int d) {
   return (size_t(BH) * n_split * Nq * d * 4 + 255) & ~size_t(255);
 }
+// Two partials per split (one per key half of the split kernel's tile).
 size_t decode_ws_bytes(int BH, int Nq, int Nkv, int d, int sms) {
   const DecodeSplit sp = decode_split(BH, Nkv, sms);
-  return decode_o_bytes(BH, sp.n_split, Nq, d) + ((size_t(BH) * sp.n_split * Nq * 2 * 4 + 255) & ~size_t(255));
+  const int n_part = 2 * sp.n_split;
+  return decode_o_bytes(BH, n_part, Nq, d) + ((size_t(BH) * n_part * Nq * 2 * 4 + 255) & ~size_t(255));
 }
 
 template <int D>
@@ -699,7 +701,7 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   if ((st = make_tile_map(&mv, v, B * H, Nkv, d, "v")) != FA_OK) return st;
   fa::DecodeParams p{};
   p.part_o = static_cast<float*>(workspace);
-  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_o_bytes(B * H, sp.n_split, Nq, d));
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_o_bytes(B * H, 2 * sp.n_split, Nq, d));
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.key_lens = key_lens;
@@ -709,6 +711,7 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   p.Nkv = Nkv;
   p.chunk = sp.chunk;
   p.n_split = sp.n_split;
+  p.n_part = 2 * sp.n_split;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_ns = g_wait_ns.load();

@@ -153,7 +153,8 @@ FA_API size_t fa_bwd_noalloc_max_scratch(void);
  * Nkv); query i is the token at position L - Nq + i, so causal keeps key j <= L - Nq + i and key
  * padding keeps j < L.  A query with no allowed key gets O = 0 and lse = -inf.  No dropout.
  * d in {64, 128}.  The key range of each head is split over CTAs (fa_fwd_decode_split splits
- * per head) that write fp32 partials (m, l, unnormalised O) into the caller's workspace (at least
+ * per head) that write fp32 partials (m, l, unnormalised O; two per split, one per key half of
+ * its 128-key blocks) into the caller's workspace (at least
  * fa_fwd_decode_workspace_size() bytes, 256-byte aligned, clobbered; not shared by calls that may
  * overlap), then a second launch merges them.  Two kernel launches.
  * The workspace size depends on the current device's SM count; with no visible device it is the
