@@ -36,6 +36,7 @@ CASES = [
     (1, 2, 1, 1, 64, False, None), (2, 2, 1, 200, 128, False, None), (1, 3, 5, 1000, 64, True, None),
     (2, 2, 16, 777, 128, True, (0, 777)), (3, 1, 8, 5000, 64, False, (3, 5000)), (1, 2, 64, 300, 128, True, None),
     (2, 1, 13, 129, 64, True, (5, 20)), (1, 4, 16, 4096, 128, False, None),
+    (2, 3, 64, 1000, 64, True, (0, 1000)), (3, 2, 1, 1, 128, True, None),
 ]
 
 
